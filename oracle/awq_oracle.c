@@ -1,0 +1,324 @@
+/*
+ * CPU oracle for the W4A16 group-quantized linear layer  y = x . dequant(Wq)^T.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is compiled into liborc.so and is used by
+ * the tests, by the smoke check and by the CPU-baseline leg of the benchmark.
+ * The product (the CUDA library) never links, loads or calls it, and it shares
+ * no code, header, table or constant generator with the CUDA path.
+ *
+ * What it computes, and the passage each step follows:
+ *   - TinyChat README, "Usage" step 3: weights are quantized to 4 bits
+ *     ("--w_bit 4") in groups of 128 input channels ("--q_group_size 128"), and
+ *     "Speed Benchmarks": the INT4 model runs as W4A16 (4-bit weights, fp16
+ *     activations).  Each weight is w = (q - z) * s with an fp16 scale s and a
+ *     4-bit zero point z per (output channel, group).
+ *   - The pages print no quantization formula.  This oracle takes the plainest
+ *     reading, asymmetric min-max over the group's raw values:
+ *         lo = min v, hi = max v, R = max(hi - lo, 1e-5)
+ *         s  = fp16_rne(R / 15)            (fp64 divide, then one fp16 rounding)
+ *         z  = clamp(rint(-lo / s), 0, 15)
+ *         q  = clamp(rint(v / s) + z, 0, 15)
+ *     with rint = round half to even, every division in fp64 against the
+ *     stored fp16 scale.
+ *   - dequant: W^[n,k] = fp16_rne((q - z) * s)  (the product is exact in fp64).
+ *   - matmul: y[m,n] = sum_k x[m,k] * W^[n,k] in fp64, in increasing k, and the
+ *     error scale B[m,n] = sum_k |x[m,k] * W^[n,k]|.
+ *   - a second, independent matmul route that factors the zero point out of
+ *     each group:  y[m,n] = sum_g s * (sum_{k in g} x*q  -  z * sum_{k in g} x).
+ *   - the packed layout (our own; the pages only name a ".pt" checkpoint):
+ *       qweight  uint32 [N/16][K/128][16][16]: block (nb, kb) holds rows
+ *                n = 16nb + r (r = 0..15) and input channels 128kb..128kb+127;
+ *                word w of row r holds k = 128kb + 8w + i, i = 0..7, with the
+ *                nibble of even i at bits 4*(i/2) and of odd i at bits
+ *                16 + 4*(i/2).  (So (word >> 4j) & 0x000F000F holds the
+ *                adjacent pair k = 8w+2j, 8w+2j+1 as two 16-bit lanes.)
+ *       scales   fp16  [K/G][N]
+ *       zeros    uint8 [K/G][N/2]: low nibble = even n, high nibble = odd n.
+ *
+ * fp16 conversions below are written from the IEEE 754 binary16 definition
+ * (1 sign bit, 5 exponent bits with bias 15, 10 fraction bits; exponent field
+ * 0 encodes subnormals f * 2^-24).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_ERR_SHAPE 2
+#define ORC_ERR_NONFINITE 8
+
+/* ------------------------------------------------------------------------- */
+/* binary16 <-> binary64                                                      */
+/* ------------------------------------------------------------------------- */
+
+double orc_half_to_double(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1F;
+  int f = h & 0x3FF;
+  double v;
+  if (e == 0)
+    v = ldexp((double)f, -24);                /* subnormal (or zero): f * 2^-24 */
+  else if (e == 31)
+    v = f ? NAN : INFINITY;
+  else
+    v = ldexp((double)(1024 + f), e - 25);    /* (1 + f/1024) * 2^(e-15) */
+  return sign ? -v : v;
+}
+
+/* Nearest binary16, ties to even, with gradual underflow and overflow to inf. */
+uint16_t orc_double_to_half(double d) {
+  uint16_t sign = signbit(d) ? 0x8000 : 0;
+  if (isnan(d)) return 0x7E00;
+  double a = fabs(d);
+  if (isinf(a) || a >= 65536.0) return sign | 0x7C00;
+  if (a == 0.0) return sign;
+  int E;
+  frexp(a, &E);          /* a = m * 2^E, m in [0.5, 1): floor(log2 a) = E - 1 */
+  int e = E - 1;
+  if (e < -14) e = -14;  /* below the normal range the spacing stays 2^-24 */
+  double quantum = ldexp(1.0, e - 10);   /* spacing of binary16 values near a */
+  double t = a / quantum;                /* exact: scaling by a power of two */
+  double r = rint(t);                    /* nearest integer, ties to even */
+  int biased = e + 15;
+  uint32_t bits;
+  if (biased == 1 && r < 1024.0) {
+    bits = (uint32_t)r;                  /* subnormal: value r * 2^-24 */
+  } else {
+    if (r >= 2048.0) { r = 1024.0; biased += 1; }  /* carry into the next binade */
+    if (biased >= 31) return sign | 0x7C00;
+    bits = ((uint32_t)biased << 10) | (uint32_t)(r - 1024.0);
+  }
+  return sign | (uint16_t)bits;
+}
+
+/* ------------------------------------------------------------------------- */
+/* quantization                                                              */
+/* ------------------------------------------------------------------------- */
+
+static int bad_shape(int64_t N, int64_t K, int G) {
+  return N <= 0 || K <= 0 || G <= 0 || K % G != 0 || K % 128 != 0 || N % 16 != 0;
+}
+
+/* Quantize one group of G values v[0..G-1] (exact fp16 values held as doubles). */
+static int quantize_group(const double* v, int G, uint8_t* q_out, uint8_t* z_out, uint16_t* s_out) {
+  double lo = v[0], hi = v[0];
+  for (int j = 0; j < G; ++j) {
+    if (!isfinite(v[j])) return ORC_ERR_NONFINITE;
+    if (v[j] < lo) lo = v[j];
+    if (v[j] > hi) hi = v[j];
+  }
+  double R = hi - lo;            /* exact: both are binary16 values */
+  if (R < 1e-5) R = 1e-5;
+  uint16_t s16 = orc_double_to_half(R / 15.0);
+  double s = orc_half_to_double(s16);
+  double z = rint(-lo / s);
+  if (z < 0.0) z = 0.0;
+  if (z > 15.0) z = 15.0;
+  for (int j = 0; j < G; ++j) {
+    double q = rint(v[j] / s) + z;
+    if (q < 0.0) q = 0.0;
+    if (q > 15.0) q = 15.0;
+    q_out[j] = (uint8_t)q;
+  }
+  *z_out = (uint8_t)z;
+  *s_out = s16;
+  return ORC_OK;
+}
+
+/* W fp16 [N][K] -> q uint8 [N][K], z uint8 [N][K/G], s fp16 [N][K/G].
+ * Returns ORC_ERR_NONFINITE if any weight is inf/NaN (the other groups are
+ * still quantized; the offending group's outputs are left untouched). */
+int orc_quantize(const uint16_t* W, int64_t N, int64_t K, int G, uint8_t* q, uint8_t* z, uint16_t* s) {
+  if (bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  int64_t ng = K / G;
+  int rc = ORC_OK;
+  double* v = (double*)malloc(sizeof(double) * (size_t)G);
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t g = 0; g < ng; ++g) {
+      for (int j = 0; j < G; ++j) v[j] = orc_half_to_double(W[n * K + g * G + j]);
+      int r = quantize_group(v, G, q + n * K + g * G, z + n * ng + g, s + n * ng + g);
+      if (r != ORC_OK) rc = r;
+    }
+  }
+  free(v);
+  return rc;
+}
+
+/* W^ fp16 [N][K] = fp16_rne((q - z) * s). */
+int orc_dequant(const uint8_t* q, const uint8_t* z, const uint16_t* s, int64_t N, int64_t K, int G,
+                uint16_t* What) {
+  if (bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  int64_t ng = K / G;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      int64_t g = k / G;
+      double sd = orc_half_to_double(s[n * ng + g]);
+      double w = ((double)q[n * K + k] - (double)z[n * ng + g]) * sd;
+      What[n * K + k] = orc_double_to_half(w);
+    }
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* packed layout                                                             */
+/* ------------------------------------------------------------------------- */
+
+/* Bit position of element i (0..7) inside its 32-bit word. */
+static int nibble_shift(int i) { return (i % 2 == 0) ? 4 * (i / 2) : 16 + 4 * (i / 2); }
+
+/* Index of the word holding (n, k) in qweight [N/16][K/128][16][16]. */
+static int64_t word_index(int64_t n, int64_t k, int64_t K) {
+  int64_t nb = n / 16, r = n % 16, kb = k / 128, w = (k % 128) / 8;
+  return ((nb * (K / 128) + kb) * 16 + r) * 16 + w;
+}
+
+int orc_pack(const uint8_t* q, const uint8_t* z, const uint16_t* s, int64_t N, int64_t K, int G,
+             uint32_t* qweight, uint16_t* scales, uint8_t* zeros) {
+  if (bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  int64_t ng = K / G;
+  memset(qweight, 0, sizeof(uint32_t) * (size_t)(N * K / 8));
+  memset(zeros, 0, (size_t)(ng * N / 2));
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k)
+      qweight[word_index(n, k, K)] |= (uint32_t)(q[n * K + k] & 0xF) << nibble_shift((int)(k % 8));
+  for (int64_t g = 0; g < ng; ++g)
+    for (int64_t n = 0; n < N; ++n) {
+      scales[g * N + n] = s[n * ng + g];
+      zeros[g * (N / 2) + n / 2] |= (uint8_t)((z[n * ng + g] & 0xF) << (4 * (n % 2)));
+    }
+  return ORC_OK;
+}
+
+int orc_unpack(const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros, int64_t N, int64_t K,
+               int G, uint8_t* q, uint8_t* z, uint16_t* s) {
+  if (bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  int64_t ng = K / G;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k)
+      q[n * K + k] = (uint8_t)((qweight[word_index(n, k, K)] >> nibble_shift((int)(k % 8))) & 0xF);
+  for (int64_t g = 0; g < ng; ++g)
+    for (int64_t n = 0; n < N; ++n) {
+      s[n * ng + g] = scales[g * N + n];
+      z[n * ng + g] = (uint8_t)((zeros[g * (N / 2) + n / 2] >> (4 * (n % 2))) & 0xF);
+    }
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* matmul                                                                    */
+/* ------------------------------------------------------------------------- */
+
+/* y[m][n] = sum_k x[m][k] * W^[n][k] (fp64, increasing k); bound = sum |.|. */
+int orc_matmul(const uint16_t* x, int64_t M, const uint16_t* What, int64_t N, int64_t K, double* y,
+               double* bound) {
+  if (M < 0 || N <= 0 || K <= 0) return ORC_ERR_SHAPE;
+  double* wd = (double*)malloc(sizeof(double) * (size_t)K);
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) wd[k] = orc_half_to_double(What[n * K + k]);
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0, b = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        double p = orc_half_to_double(x[m * K + k]) * wd[k];
+        acc += p;
+        b += fabs(p);
+      }
+      y[m * N + n] = acc;
+      if (bound) bound[m * N + n] = b;
+    }
+  }
+  free(wd);
+  return ORC_OK;
+}
+
+/* Second route: zero point factored out of each group. */
+int orc_matmul_factored(const uint16_t* x, int64_t M, const uint8_t* q, const uint8_t* z, const uint16_t* s,
+                        int64_t N, int64_t K, int G, double* y) {
+  if (M < 0 || bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  int64_t ng = K / G;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int64_t g = 0; g < ng; ++g) {
+        double sxq = 0.0, sx = 0.0;
+        for (int j = 0; j < G; ++j) {
+          double xv = orc_half_to_double(x[m * K + g * G + j]);
+          sxq += xv * (double)q[n * K + g * G + j];
+          sx += xv;
+        }
+        acc += orc_half_to_double(s[n * ng + g]) * (sxq - (double)z[n * ng + g] * sx);
+      }
+      y[m * N + n] = acc;
+    }
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* the whole linear layer from the packed buffers                            */
+/* ------------------------------------------------------------------------- */
+
+/* Dequantized row n of the packed weight: W^[n][0..K). */
+static void packed_row(const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros, int64_t N,
+                       int64_t K, int G, int64_t n, double* row) {
+  for (int64_t k = 0; k < K; ++k) {
+    int64_t g = k / G;
+    uint32_t q = (qweight[word_index(n, k, K)] >> nibble_shift((int)(k % 8))) & 0xF;
+    uint32_t z = (zeros[g * (N / 2) + n / 2] >> (4 * (n % 2))) & 0xF;
+    double s = orc_half_to_double(scales[g * N + n]);
+    row[k] = orc_half_to_double(orc_double_to_half(((double)q - (double)z) * s));
+  }
+}
+
+/* y, bound [M][n1-n0]: output channels n0..n1-1 of x . W^T, straight from the
+ * packed buffers (unpack, dequant, fp64 dot products). */
+int orc_linear_rows(const uint16_t* x, int64_t M, const uint32_t* qweight, const uint16_t* scales,
+                    const uint8_t* zeros, int64_t N, int64_t K, int G, int64_t n0, int64_t n1, double* y,
+                    double* bound) {
+  if (M < 0 || bad_shape(N, K, G) || n0 < 0 || n1 > N || n0 > n1) return ORC_ERR_SHAPE;
+  int64_t W = n1 - n0;
+  double* row = (double*)malloc(sizeof(double) * (size_t)K);
+  for (int64_t n = n0; n < n1; ++n) {
+    packed_row(qweight, scales, zeros, N, K, G, n, row);
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0, b = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        double p = orc_half_to_double(x[m * K + k]) * row[k];
+        acc += p;
+        b += fabs(p);
+      }
+      y[m * W + (n - n0)] = acc;
+      if (bound) bound[m * W + (n - n0)] = b;
+    }
+  }
+  free(row);
+  return ORC_OK;
+}
+
+int orc_linear(const uint16_t* x, int64_t M, const uint32_t* qweight, const uint16_t* scales,
+               const uint8_t* zeros, int64_t N, int64_t K, int G, double* y, double* bound) {
+  return orc_linear_rows(x, M, qweight, scales, zeros, N, K, G, 0, N, y, bound);
+}
+
+/* Individual outputs (ms[i], ns[i]) of x . W^T from the packed buffers. */
+int orc_linear_entries(const uint16_t* x, int64_t M, const uint32_t* qweight, const uint16_t* scales,
+                       const uint8_t* zeros, int64_t N, int64_t K, int G, const int64_t* ms,
+                       const int64_t* ns, int64_t count, double* y, double* bound) {
+  if (M < 0 || bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  double* row = (double*)malloc(sizeof(double) * (size_t)K);
+  int64_t cached = -1;
+  for (int64_t i = 0; i < count; ++i) {
+    int64_t m = ms[i], n = ns[i];
+    if (m < 0 || m >= M || n < 0 || n >= N) { free(row); return ORC_ERR_SHAPE; }
+    if (n != cached) { packed_row(qweight, scales, zeros, N, K, G, n, row); cached = n; }
+    double acc = 0.0, b = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+      double p = orc_half_to_double(x[m * K + k]) * row[k];
+      acc += p;
+      b += fabs(p);
+    }
+    y[i] = acc;
+    if (bound) bound[i] = b;
+  }
+  free(row);
+  return ORC_OK;
+}
