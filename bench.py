@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 group-quantized linear layer on B200.
+
+One step = one decode pass over the LLaMA-2-7B decoder-layer linear set at
+M = 1 (qkv 4096->12288, o_proj 4096->4096, gate_up 4096->22016,
+down 11008->4096; group 128), i.e. four awq_linear calls, each a W4A16 GEMV
+that streams its packed weights from HBM once. Inputs are seeded synthetic
+(weights ~ N(0, 0.02), activations ~ N(0, 1)), quantized and packed on the
+GPU by awq_pack before timing. Six rotating copies of the packed weights
+(6 x 105 MB, more than the 126 MB L2) make every step read HBM.
+
+Prints ONE JSON line (rank 0): the metric (GB/s of algorithmic bytes, whole
+job), the roofline of the GEMV kernel, an end-to-end figure through the
+public API with host buffers, the CPU oracle baseline, the clocks seen
+during the timed region, and a secondary prefill GEMM figure (TFLOP/s).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  torchrun --nproc-per-node N bench.py --gpus N ...   (N independent replicas)
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import awq_synth  # noqa: E402
+
+WORKLOAD = "llama2_7b_decode"
+M_DECODE = 1
+ROTATIONS = 6
+PREFILL = ("prefill", "llama3_gate_up", 2048)
+METRIC = "W4A16 decode GEMV GB/s (% of HBM peak); prefill GEMM TFLOP/s (% tensor peak)"
+GEMV_SRC = os.path.join(ROOT, "weight_only_bit_awq_b200", "csrc", "gemv.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_llama2_7b_decode_traffic.json")
+
+
+def algo_bytes(M, K, N, group=128):
+    """Bytes a W4A16 linear call must move: packed weight, scales, zeros, x, y."""
+    return K * N // 2 + 2 * (K // group) * N + (K // group) * N // 2 + 2 * M * K + 2 * M * N
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_per_launch():
+    """Mean DRAM bytes per GEMV launch from the committed ncu capture, or None
+    if the GEMV source changed since it was taken."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    h = hashlib.sha256(open(GEMV_SRC, "rb").read()).hexdigest()
+    if d.get("gemv_src_sha256") != h:
+        return None
+    return d.get("dram_bytes_per_step", 0) / max(1, d.get("launches_per_step", 1))
+
+
+# --------------------------------------------------------------------------
+# reference arm: the CPU oracle as it stands, on host cores
+# --------------------------------------------------------------------------
+
+def cpu_oracle_step(layers_packed, xs, frac):
+    """One step of the workload through the oracle, on the first `frac` of
+    every layer's output channels. Returns (algorithmic bytes covered, seconds)."""
+    import oracle
+    t0 = time.perf_counter()
+    tot = 0.0
+    for (L, hp), x in zip(layers_packed, xs):
+        n1 = max(16, int(L.N * frac) // 16 * 16)
+        oracle.linear(x, *hp, L.N, L.K, rows=(0, n1))
+        tot += algo_bytes(M_DECODE, L.K, L.N) * n1 / L.N
+    return tot, time.perf_counter() - t0
+
+
+def host_workload(rows=None, seed=0):
+    """Oracle-packed weights of the workload's layers (all rows, or the first `rows`)."""
+    import oracle
+    wl = awq_synth.WORKLOADS[WORKLOAD]
+    out, xs = [], []
+    for L in wl.layers:
+        W = awq_synth.layer_weight(seed, wl, L, rows=None if rows is None else slice(0, rows))
+        n = W.shape[0]
+        Ls = awq_synth.Layer(L.name, L.K, n)
+        out.append((Ls, oracle.quantize_pack(W), L))
+        xs.append(awq_synth.layer_input(seed, wl, L, M_DECODE))
+    return wl, out, xs
+
+
+def run_reference(args):
+    """The oracle, as it stands, timed on the host cores. Each step is a
+    bounded sample of the workload: `rows_per_step` output channels taken
+    round-robin from the first 64 rows of the four layers, sized so that
+    warm-up plus timed steps take about --ref-budget seconds."""
+    import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl, pool, xs = host_workload(rows=64)
+    order = [(li, r) for r in range(64) for li in range(len(pool))]
+    t0 = time.perf_counter()
+    for li in range(len(pool)):
+        Ls, hp, L = pool[li]
+        oracle.linear(xs[li], *hp, Ls.N, Ls.K, rows=(0, 1))
+    t_row = (time.perf_counter() - t0) / len(pool)
+    rows_per_step = int(max(1, min(len(order), args.ref_budget / (args.steps + args.warmup) / t_row)))
+    cursor = 0
+
+    def one_step():
+        nonlocal cursor
+        b = 0.0
+        t = time.perf_counter()
+        for _ in range(rows_per_step):
+            li, r = order[cursor % len(order)]
+            cursor += 1
+            Ls, hp, L = pool[li]
+            oracle.linear(xs[li], *hp, Ls.N, Ls.K, rows=(r, r + 1))
+            b += algo_bytes(M_DECODE, L.K, L.N) / L.N
+        return b, time.perf_counter() - t
+
+    for _ in range(args.warmup):
+        one_step()
+    tot_b, tot_t = 0.0, 0.0
+    for _ in range(args.steps):
+        b, t = one_step()
+        tot_b += b
+        tot_t += t
+    gbs = tot_b / tot_t / 1e9
+    sample = (f"{rows_per_step} output channel(s) per step, round-robin over the first 64 rows of the four "
+              f"layers (fp64 C oracle: unpack, dequant, dot products; single thread)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M_DECODE, "group": 128,
+                   "layers": [[L.name, L.K, L.N] for L in wl.layers]},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import weight_only_bit_awq_b200 as awq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    hbm, tc_burst, tc_sus, peak_kind = peaks()
+    wl = awq_synth.WORKLOADS[WORKLOAD]
+    layers = wl.layers
+    ws = awq.new_workspace(M_DECODE, max(L.K for L in layers), max(L.N for L in layers), dev)
+    ws_bytes = max(awq.awq_workspace_bytes(M_DECODE, L.K, L.N) for L in layers)
+    if ws.numel() < ws_bytes:
+        ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+
+    # inputs: seeded weights, packed on this GPU by awq_pack (K1), R copies
+    packed = [[] for _ in range(ROTATIONS)]
+    xs, ys = [], []
+    for L in layers:
+        W = torch.from_numpy(awq_synth.layer_weight(0, wl, L).view(np.uint16)).view(torch.float16).to(dev)
+        qw, sc, ze = awq.awq_pack(W, ws)
+        st = awq.awq_get_status(ws)
+        if st != awq.AWQ_OK:
+            raise RuntimeError(awq.awq_status_string(st))
+        del W
+        for r in range(ROTATIONS):
+            packed[r].append((qw.clone(), sc.clone(), ze.clone()) if r else (qw, sc, ze))
+        x = torch.from_numpy(awq_synth.layer_input(0, wl, L, M_DECODE).view(np.uint16)).view(torch.float16).to(dev)
+        xs.append(x)
+        ys.append(torch.empty((M_DECODE, L.N), dtype=torch.float16, device=dev))
+    step_bytes = sum(algo_bytes(M_DECODE, L.K, L.N) for L in layers)
+
+    def step(r):
+        for L, x, y, (qw, sc, ze) in zip(layers, xs, ys, packed[r]):
+            awq.awq_linear(x, qw, sc, ze, L.N, ws, y=y)
+
+    # CUDA graphs: one graph per rotation copy (one step = 4 kernel launches)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        for r in range(ROTATIONS):   # warm the launch paths before capture
+            step(r)
+    torch.cuda.synchronize()
+    graphs = []
+    for r in range(ROTATIONS):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(r)
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % ROTATIONS].replay()
+    barrier()
+    st = awq.awq_get_status(ws)
+    if st != awq.AWQ_OK:
+        raise RuntimeError(awq.awq_status_string(st))
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for i in range(args.steps):
+                graphs[i % ROTATIONS].replay()
+            ev1.record(stream)
+        barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    clocks = clk.summary()
+    st = awq.awq_get_status(ws)
+    if st != awq.AWQ_OK:
+        raise RuntimeError(awq.awq_status_string(st))
+    value = step_bytes * args.steps * world / (ms * 1e-3) / 1e9
+    per_gpu_gbs = step_bytes * args.steps / (ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API with pinned host buffers ----
+    xh = [torch.empty_like(x, device="cpu").pin_memory().copy_(x.cpu()) for x in xs]
+    yh = [torch.empty_like(y, device="cpu").pin_memory() for y in ys]
+    e2e_steps = max(3, min(args.steps, 2000))
+
+    def e2e_step(r):
+        for L, xhst, x, y, yhst, (qw, sc, ze) in zip(layers, xh, xs, ys, yh, packed[r]):
+            x.copy_(xhst, non_blocking=True)
+            awq.awq_linear(x, qw, sc, ze, L.N, ws, y=y)
+            yhst.copy_(y, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            e2e_step(i % ROTATIONS)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i % ROTATIONS)
+        e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e = {"value": step_bytes * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": sum(x.numel() * 2 for x in xs),
+           "d2h_bytes_per_step": sum(y.numel() * 2 for y in ys),
+           "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
+
+    # ---- secondary: prefill GEMM on the tensor cores ----
+    prefill = None
+    if not args.no_prefill:
+        pwl = awq_synth.WORKLOADS[PREFILL[0]]
+        PL = pwl.layer(PREFILL[1])
+        Mp = PREFILL[2]
+        W = torch.from_numpy(awq_synth.layer_weight(0, pwl, PL).view(np.uint16)).view(torch.float16).to(dev)
+        pws = awq.new_workspace(Mp, PL.K, PL.N, dev)
+        pq = awq.awq_pack(W, pws)
+        del W
+        xp = torch.from_numpy(awq_synth.layer_input(0, pwl, PL, Mp).view(np.uint16)).view(torch.float16).to(dev)
+        yp = torch.empty((Mp, PL.N), dtype=torch.float16, device=dev)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                awq.awq_linear(xp, *pq, PL.N, pws, y=yp)
+        torch.cuda.synchronize()
+        reps = 20
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            p0.record(stream)
+            for _ in range(reps):
+                awq.awq_linear(xp, *pq, PL.N, pws, y=yp)
+            p1.record(stream)
+        torch.cuda.synchronize()
+        st = awq.awq_get_status(pws)
+        if st != awq.AWQ_OK:
+            raise RuntimeError(awq.awq_status_string(st))
+        pms = max_over_ranks(p0.elapsed_time(p1)) / reps
+        tflops = 2.0 * Mp * PL.N * PL.K / (pms * 1e-3) / 1e12
+        prefill = {"workload": f"{PREFILL[1]} K={PL.K} N={PL.N} M={Mp}", "ms": pms, "tflops_per_gpu": tflops,
+                   "peak_tflops": tc_burst, "frac": tflops / tc_burst, "peak_kind": f"{peak_kind} bf16 burst"}
+
+    # ---- CPU oracle baseline on a bounded sample (rank 0, N = 1 only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        _, hl, hx = host_workload()
+        b, t = cpu_oracle_step([(L, hp) for L, hp, _ in hl], hx, args.cpu_frac)
+        cpu = {"value": b / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"one step on the first {args.cpu_frac:.3f} of each layer's output channels "
+                         f"({t:.1f} s, fp64 C oracle, single thread)"}
+
+    traffic = traffic_per_launch()
+    launches = len(layers) * args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M_DECODE, "group": 128,
+                   "layers": [[L.name, L.K, L.N] for L in layers],
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"{ROTATIONS} rotating packed-weight copies ({ROTATIONS * step_bytes / 1e6:.0f} MB > 126 MB L2)",
+                   "timing": "CUDA graphs, one graph per step, CUDA events on the replay stream"},
+        "roofline": {"bound": "hbm", "achieved": per_gpu_gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": per_gpu_gbs / hbm, "traffic": traffic,
+                     "kernel": "gemv_kernel (awq_w4a16_gemv via awq_linear)",
+                     "peak_kind": f"{peak_kind} HBM copy"},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "prefill_gemm": prefill,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in graphs:
+        del g
+    graphs.clear()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-frac", type=float, default=1.0, help="share of rows in the CPU-baseline sample")
+    ap.add_argument("--ref-budget", type=float, default=60.0, help="seconds of oracle work in the reference arm")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,156 @@
+/*
+ * awq.h -- C ABI of libawq_b200.so: W4A16 group-quantized linear layer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (TinyChat: Efficient and Lightweight Chatbot with AWQ,
+ * README sections "Speed Benchmarks" and "Usage", step 3):
+ *   weights are stored as 4-bit unsigned codes q with one fp16 scale s and one
+ *   4-bit zero point z per (output channel, group of 128 input channels)
+ *   ("--w_bit 4 --q_group_size 128"), each weight is w = (q - z) * s, and the
+ *   layer runs as W4A16: fp16 activations times 4-bit weights, fp16 output.
+ *
+ *   y[m][n] = sum_k x[m][k] * W^[n][k],   W^[n][k] = fp16_rne((q - z) * s)
+ *
+ * Orientation: W is [N][K] (N output channels, K input channels, K
+ * contiguous), x is [M][K] and y is [M][N], all row-major.
+ *
+ * ---------------------------------------------------------------------------
+ * Packed layout (ours; the README names only a "-w4-g128-awq.pt" checkpoint)
+ * ---------------------------------------------------------------------------
+ *   qweight  uint32 [N/16][K/128][16][16]   (K*N/2 bytes)
+ *            Block (nb, kb) is 1 KiB, holds output channels n = 16*nb + r
+ *            (r = 0..15) and input channels 128*kb .. 128*kb + 127. Word w of
+ *            row r holds k = 128*kb + 8*w + i for i = 0..7: the code of even i
+ *            at bits 4*(i/2) .. 4*(i/2)+3 and the code of odd i at bits
+ *            16 + 4*(i/2) .. 16 + 4*(i/2)+3. So (word >> 4*j) & 0x000F000F
+ *            holds the adjacent pair k = 8w + 2j, 8w + 2j + 1 as two 16-bit
+ *            lanes, and a 16x128 tile is one contiguous 1 KiB load.
+ *   scales   fp16  [K/group][N]             (2*N*K/group bytes)
+ *   zeros    uint8 [K/group][N/2]           (N*K/(2*group) bytes): the zero
+ *            point of even n in the low nibble, of odd n in the high nibble.
+ *
+ * Quantization (awq_pack), per (n, group) over the group's raw values v:
+ *   lo = min v, hi = max v, R = max(hi - lo, 1e-5)
+ *   s = fp16_rne(R / 15), z = clamp(rint(-lo / s), 0, 15),
+ *   q = clamp(rint(v / s) + z, 0, 15)
+ * with every division in fp64 against the stored fp16 s and rint rounding
+ * half to even. The pages print no formula; this is the plainest reading of
+ * asymmetric min-max 4-bit quantization with fp16 scales and 4-bit zeros.
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions for every entry point
+ * ---------------------------------------------------------------------------
+ *   Shapes     M >= 0 (M = 0 is a no-op), K > 0 and K % 128 == 0, N > 0 and
+ *              N % 16 == 0, group == 128 (else AWQ_ERR_UNSUPPORTED).
+ *   Pointers   device pointers unless stated; all non-null (x and y may be
+ *              null when M == 0) and 16-byte aligned (AWQ_ERR_INVALID_ARG /
+ *              AWQ_ERR_ALIGNMENT). Outputs may not overlap inputs.
+ *   Ownership  the caller allocates and owns every buffer, the workspace
+ *              included. The library allocates no device memory; it keeps
+ *              only per-device launch parameters (SM count, kernel attributes).
+ *   Streams    `stream` is a cudaStream_t (NULL = legacy default stream).
+ *              Calls are asynchronous on it; only awq_get_status synchronizes.
+ *   Errors     argument errors are returned before anything is launched;
+ *              AWQ_ERR_CUDA reports a failed launch. Errors found on the device
+ *              (a non-finite weight in awq_pack, a bounded wait that expired)
+ *              are recorded in the workspace status word and read back with
+ *              awq_get_status.
+ *   Workspace  at least awq_workspace_bytes(M, K, N, group) bytes of device
+ *              memory, zeroed once with awq_workspace_init before first use.
+ *              Kernels leave it zeroed again (split-K counters reset
+ *              themselves). One workspace must not be used by two calls that
+ *              can run at the same time (e.g. on two streams).
+ */
+#ifndef AWQ_B200_H
+#define AWQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum awq_status {
+  AWQ_OK = 0,
+  AWQ_ERR_INVALID_ARG = 1, /* null pointer, overlapping buffers, bad workspace */
+  AWQ_ERR_SHAPE = 2,       /* M < 0, K <= 0, N <= 0, K % 128, N % 16, K % group */
+  AWQ_ERR_ALIGNMENT = 3,   /* a pointer that is not 16-byte aligned */
+  AWQ_ERR_WORKSPACE = 4,   /* ws_bytes below awq_workspace_bytes(...) */
+  AWQ_ERR_UNSUPPORTED = 5, /* group != 128, M above an entry's limit, no sm_100 device */
+  AWQ_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed */
+  AWQ_ERR_TIMEOUT = 7,     /* device side: a bounded pipeline wait expired */
+  AWQ_ERR_NONFINITE = 8    /* device side: awq_pack met an inf or NaN weight */
+} awq_status;
+
+typedef struct awq_packed_sizes {
+  size_t qweight_bytes; /* K*N/2 */
+  size_t scales_bytes;  /* 2*N*(K/group) */
+  size_t zeros_bytes;   /* N*(K/group)/2 */
+} awq_packed_sizes;
+
+/* Largest M accepted by awq_w4a16_gemv (the decode path). */
+#define AWQ_GEMV_MAX_M 32
+
+/* Sizes of the three packed buffers for a [N][K] weight. Host only.
+ * Returns AWQ_ERR_SHAPE / AWQ_ERR_UNSUPPORTED / AWQ_ERR_INVALID_ARG (out NULL). */
+awq_status awq_packed_size(int64_t K, int64_t N, int group, awq_packed_sizes* out);
+
+/* Workspace bytes needed by any entry point below for these sizes on the
+ * current device (split-K partials, counters, the status word). Host only.
+ * Returns 0 for invalid sizes. */
+size_t awq_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
+
+/* Zero `ws_bytes` bytes of workspace on `stream` (needed once, before the
+ * first use of a new workspace). */
+awq_status awq_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* Quantize and pack (TinyChat README, Usage step 3: "--w_bit 4
+ * --q_group_size 128 ... --q_backend real"): W fp16 [N][K] -> qweight,
+ * scales, zeros in the layout above, bit for bit the quantization stated
+ * above. An inf/NaN weight records AWQ_ERR_NONFINITE in the workspace status
+ * word (its group's outputs are then unspecified). */
+awq_status awq_pack(const void* w, int64_t K, int64_t N, int group, void* qweight, void* scales, void* zeros,
+                    void* workspace, size_t ws_bytes, void* stream);
+
+/* Dequantize: W^ fp16 [N][K] = fp16_rne((q - z) * s) for every (n, k). */
+awq_status awq_dequant(const void* qweight, const void* scales, const void* zeros, int64_t K, int64_t N,
+                       int group, void* w_out, void* stream);
+
+/* Decode-stage W4A16 GEMV, 1 <= M <= AWQ_GEMV_MAX_M (README "Speed
+ * Benchmarks": per-token latency of the generation stage): y fp16 [M][N] =
+ * x fp16 [M][K] . W^T. Streams the packed weights once; fp32 accumulation.
+ * M > AWQ_GEMV_MAX_M returns AWQ_ERR_UNSUPPORTED. */
+awq_status awq_w4a16_gemv(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
+                          int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,
+                          void* stream);
+
+/* Context-stage (prefill) W4A16 GEMM for any M (README "New Optimization of
+ * Context Stage": the prompt is processed as one batch of tokens): same
+ * result as awq_w4a16_gemv, on the tcgen05 tensor cores with fp32
+ * accumulation in tensor memory. */
+awq_status awq_w4a16_gemm(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
+                          int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,
+                          void* stream);
+
+/* The linear layer: awq_w4a16_gemv for M <= awq_linear_gemv_limit(), else
+ * awq_w4a16_gemm. */
+awq_status awq_linear(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
+                      int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,
+                      void* stream);
+
+/* The M at and below which awq_linear takes the GEMV path. */
+int awq_linear_gemv_limit(void);
+
+/* Synchronize `stream`, then return and clear the device-side status word of
+ * `workspace` (AWQ_OK if no device-side error was recorded). */
+awq_status awq_get_status(void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* awq_status_string(awq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_B200_H */

@@ -1,0 +1,122 @@
+"""The C ABI library on the host: it loads, exports every symbol include/awq.h
+declares, and rejects bad arguments with the documented codes before anything
+is launched. No test here launches a kernel: the pointers are fake, and the
+only call that gets past the argument checks runs only when no GPU exists
+(it must then stop at the device check)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import weight_only_bit_awq_b200 as awq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "awq.h")
+L = awq.lib
+
+FAKE = 0x7F0000000000          # 16-byte aligned, never dereferenced
+FAKE2 = FAKE + (1 << 32)
+FAKE3 = FAKE + (2 << 32)
+FAKE4 = FAKE + (3 << 32)
+FAKE5 = FAKE + (4 << 32)
+FAKE6 = FAKE + (5 << 32)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:awq_status|size_t|int|const char\*)\s+(awq_\w+)\(", text, re.M)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(awq.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        ctypes.cast(getattr(L, name), ctypes.c_void_p)
+
+
+def test_status_strings():
+    for code, name in awq.STATUS_NAMES.items():
+        assert awq.awq_status_string(code).startswith(name)
+    assert "unknown" in awq.awq_status_string(99)
+
+
+def test_packed_sizes():
+    assert awq.awq_packed_size(4096, 4096) == (4096 * 4096 // 2, 4096 // 128 * 4096 * 2, 4096 // 128 * 4096 // 2)
+    assert awq.awq_packed_size(11008, 4096)[0] == 11008 * 4096 // 2
+
+
+@pytest.mark.parametrize("K,N,group,code", [
+    (100, 16, 128, awq.AWQ_ERR_SHAPE), (128, 15, 128, awq.AWQ_ERR_SHAPE), (0, 16, 128, awq.AWQ_ERR_SHAPE),
+    (128, 0, 128, awq.AWQ_ERR_SHAPE), (-128, 16, 128, awq.AWQ_ERR_SHAPE), (192, 16, 128, awq.AWQ_ERR_SHAPE),
+    (128, 16, 64, awq.AWQ_ERR_UNSUPPORTED), (128, 16, 32, awq.AWQ_ERR_UNSUPPORTED),
+    (1 << 23, 16, 128, awq.AWQ_ERR_UNSUPPORTED),
+])
+def test_packed_size_rejects(K, N, group, code):
+    with pytest.raises(awq.AwqError) as e:
+        awq.awq_packed_size(K, N, group)
+    assert e.value.status == code
+
+
+def test_workspace_bytes():
+    assert awq.awq_workspace_bytes(1, 100, 16) == 0
+    assert awq.awq_workspace_bytes(-1, 128, 16) == 0
+    assert awq.awq_workspace_bytes(0, 4096, 4096) >= 256
+    assert awq.awq_workspace_bytes(2048, 4096, 4096) >= 256
+    # the decode path's split-K partials grow with M * N
+    assert awq.awq_workspace_bytes(32, 4096, 4096) >= awq.awq_workspace_bytes(1, 4096, 4096)
+
+
+def _linear(fn, x=FAKE, q=FAKE2, s=FAKE3, z=FAKE4, y=FAKE5, M=1, K=4096, N=4096, group=128, ws=FAKE6,
+            ws_bytes=1 << 30):
+    return getattr(L, fn)(x, q, s, z, y, M, K, N, group, ws, ws_bytes, None)
+
+
+ENTRIES = ["awq_w4a16_gemv", "awq_w4a16_gemm", "awq_linear"]
+
+
+@pytest.mark.parametrize("fn", ENTRIES)
+def test_linear_argument_errors(fn):
+    assert _linear(fn, M=-1) == awq.AWQ_ERR_SHAPE
+    assert _linear(fn, K=4000) == awq.AWQ_ERR_SHAPE
+    assert _linear(fn, N=4104) == awq.AWQ_ERR_SHAPE
+    assert _linear(fn, group=64) == awq.AWQ_ERR_UNSUPPORTED
+    assert _linear(fn, x=None) == awq.AWQ_ERR_INVALID_ARG
+    assert _linear(fn, y=None) == awq.AWQ_ERR_INVALID_ARG
+    assert _linear(fn, ws=None) == awq.AWQ_ERR_INVALID_ARG
+    assert _linear(fn, x=FAKE + 8) == awq.AWQ_ERR_ALIGNMENT
+    assert _linear(fn, z=FAKE4 + 2) == awq.AWQ_ERR_ALIGNMENT
+    assert _linear(fn, y=FAKE + 16) == awq.AWQ_ERR_INVALID_ARG          # y overlaps x
+    assert _linear(fn, ws_bytes=16) == awq.AWQ_ERR_WORKSPACE
+    assert _linear(fn, M=0) == awq.AWQ_OK                                  # empty batch: nothing to do
+    assert _linear(fn, M=0, x=None, y=None) == awq.AWQ_OK                  # ... and x, y may be null
+
+
+def test_gemv_rejects_large_batches():
+    assert _linear("awq_w4a16_gemv", M=33) == awq.AWQ_ERR_UNSUPPORTED
+
+
+def test_pack_and_dequant_argument_errors():
+    assert L.awq_pack(FAKE, 100, 4096, 128, FAKE2, FAKE3, FAKE4, FAKE5, 1 << 20, None) == awq.AWQ_ERR_SHAPE
+    assert L.awq_pack(None, 4096, 4096, 128, FAKE2, FAKE3, FAKE4, FAKE5, 1 << 20, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_pack(FAKE + 2, 4096, 4096, 128, FAKE2, FAKE3, FAKE4, FAKE5, 1 << 20, None) == awq.AWQ_ERR_ALIGNMENT
+    assert L.awq_pack(FAKE, 4096, 4096, 128, FAKE, FAKE3, FAKE4, FAKE5, 1 << 20, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_pack(FAKE, 4096, 4096, 128, FAKE2, FAKE3, FAKE4, FAKE5, 8, None) == awq.AWQ_ERR_WORKSPACE
+    assert L.awq_pack(FAKE, 4096, 4096, 64, FAKE2, FAKE3, FAKE4, FAKE5, 1 << 20, None) == awq.AWQ_ERR_UNSUPPORTED
+    assert L.awq_dequant(FAKE2, FAKE3, FAKE4, 4096, 4096, 128, None, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_dequant(FAKE2, FAKE3, FAKE4, 4096, 4095, 128, FAKE, None) == awq.AWQ_ERR_SHAPE
+    assert L.awq_dequant(FAKE2, FAKE3, FAKE4 + 1, 4096, 4096, 128, FAKE, None) == awq.AWQ_ERR_ALIGNMENT
+    assert L.awq_workspace_init(None, 256, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_get_status(None, None) == awq.AWQ_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="would launch with fake pointers on a GPU")
+def test_valid_arguments_without_a_device_stop_at_the_device_check():
+    for fn in ENTRIES:
+        assert _linear(fn) == awq.AWQ_ERR_UNSUPPORTED
+    assert L.awq_pack(FAKE, 4096, 4096, 128, FAKE2, FAKE3, FAKE4, FAKE5, 1 << 20, None) == awq.AWQ_ERR_UNSUPPORTED
+    assert L.awq_dequant(FAKE2, FAKE3, FAKE4, 4096, 4096, 128, FAKE, None) == awq.AWQ_ERR_UNSUPPORTED

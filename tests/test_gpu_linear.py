@@ -1,0 +1,172 @@
+"""GPU W4A16 GEMV / GEMM / linear against the fp64 oracle, element by element
+within |y - y_ref| <= 2e-3 * sum|x w| + 1e-3, on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import awq_synth
+import oracle
+import weight_only_bit_awq_b200 as awq
+from gpu_helpers import (check_close, gpu_pack, host, layer_inputs, oracle_rows, packed_to_host, sample_rows,
+                         to_dev)
+
+pytestmark = pytest.mark.gpu
+G = 128
+
+
+def _packed(N, K, tag, std=0.02):
+    W = awq_synth.matrix_f16(awq_synth.key(0, 96, f"{tag}/W"), N, K, std)
+    dev = gpu_pack(W)
+    return W, dev, packed_to_host(*dev)
+
+
+def _run(fn, x, dev, N, M=None):
+    xd = to_dev(x.view(np.uint16), torch.float16)
+    M = x.shape[0]
+    K = x.shape[1]
+    ws = awq.new_workspace(M, K, N, xd.device)
+    y = fn(xd, *dev, N, ws)
+    st = awq.awq_get_status(ws)
+    assert st == awq.AWQ_OK, awq.awq_status_string(st)
+    return host(y, np.float16)
+
+
+# small and ragged shapes: several row blocks and k-blocks, N not a multiple
+# of the 128-row GEMM tile, single-k-block K, split-K on and off
+SHAPES = [(128, 16), (256, 48), (384, 336), (1024, 592), (2048, 4096), (4096, 272), (11008, 160)]
+
+
+@pytest.mark.parametrize("K,N", SHAPES)
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 9, 16, 17, 31, 32])
+def test_gemv_matches_oracle(K, N, M):
+    W, dev, hp = _packed(N, K, f"gemv{K}x{N}")
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"gemv{K}x{N}/x{M}"), M, K, 1.0)
+    y = _run(awq.awq_w4a16_gemv, x, dev, N)
+    y_ref, b = oracle.linear(x, *hp, N, K)
+    check_close(y, y_ref, b, f"gemv M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("K,N", SHAPES)
+@pytest.mark.parametrize("M", [1, 7, 64, 128, 129, 200, 256, 257, 513])
+def test_gemm_matches_oracle(K, N, M):
+    W, dev, hp = _packed(N, K, f"gemm{K}x{N}")
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"gemm{K}x{N}/x{M}"), M, K, 1.0)
+    y = _run(awq.awq_w4a16_gemm, x, dev, N)
+    y_ref, b = oracle.linear(x, *hp, N, K)
+    check_close(y, y_ref, b, f"gemm M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("fn", [awq.awq_w4a16_gemv, awq.awq_w4a16_gemm])
+def test_one_hot_activations_give_the_dequantized_weight_exactly(fn):
+    K, N = 512, 336
+    W, dev, hp = _packed(N, K, "onehot")
+    ks = [0, 1, 7, 127, 128, 300, 511, 64]
+    x = np.zeros((len(ks), K), np.float16)
+    for m, k in enumerate(ks):
+        x[m, k] = 1.0
+    y = _run(fn, x, dev, N)
+    q, z, s = oracle.unpack(*hp, N, K)
+    wh = oracle.dequant(q, z, s)
+    for m, k in enumerate(ks):
+        assert (y[m].view(np.uint16) == wh[:, k].view(np.uint16)).all(), (fn.__name__, k)
+
+
+def test_linear_dispatch_and_empty_batch():
+    K, N = 1024, 256
+    W, dev, hp = _packed(N, K, "disp")
+    lim = awq.awq_linear_gemv_limit()
+    for M in (1, lim, lim + 1, 300):
+        x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"disp/x{M}"), M, K, 1.0)
+        y = _run(awq.awq_linear, x, dev, N)
+        y_ref, b = oracle.linear(x, *hp, N, K)
+        check_close(y, y_ref, b, f"linear M={M}")
+    x0 = torch.empty((0, K), dtype=torch.float16, device="cuda")
+    ws = awq.new_workspace(0, K, N, x0.device)
+    for fn in (awq.awq_linear, awq.awq_w4a16_gemv, awq.awq_w4a16_gemm):
+        assert fn(x0, *dev, N, ws).shape == (0, N)
+
+
+def test_split_k_is_deterministic_and_the_workspace_reusable():
+    K, N = 11008, 4096
+    W, dev, hp = _packed(N, K, "det")
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, "det/x"), 3, K, 1.0)
+    xd = to_dev(x.view(np.uint16), torch.float16)
+    ws = awq.new_workspace(3, K, N, xd.device)
+    ys = [host(awq.awq_w4a16_gemv(xd, *dev, N, ws), np.uint16) for _ in range(3)]
+    assert (ys[0] == ys[1]).all() and (ys[1] == ys[2]).all()
+    # counters were left at zero: the tail of the workspace holds no stale state
+    assert awq.awq_get_status(ws) == awq.AWQ_OK
+
+
+def test_gemv_and_gemm_agree_closely():
+    K, N, M = 4096, 1024, 16
+    W, dev, hp = _packed(N, K, "agree")
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, "agree/x"), M, K, 1.0)
+    y1 = _run(awq.awq_w4a16_gemv, x, dev, N).astype(np.float64)
+    y2 = _run(awq.awq_w4a16_gemm, x, dev, N).astype(np.float64)
+    y_ref, b = oracle.linear(x, *hp, N, K)
+    check_close(y1, y_ref, b)
+    check_close(y2, y_ref, b)
+
+
+# ---- full-size workloads, sampled against the oracle ----------------------
+
+DECODE_CASES = [("single_4096", "linear", 1)]
+DECODE_CASES += [("llama2_7b_decode", l.name, 1) for l in awq_synth.WORKLOADS["llama2_7b_decode"].layers]
+DECODE_CASES += [("llama3_8b_decode", l.name, M) for l in awq_synth.WORKLOADS["llama3_8b_decode"].layers
+                 for M in (1, 4, 8, 16, 32)]
+DECODE_CASES += [("llama2_70b_decode", l.name, M) for l in awq_synth.WORKLOADS["llama2_70b_decode"].layers
+                 for M in (1, 8, 32)]
+
+
+_cache = {}
+
+
+def _full_layer(wl, layer):
+    key = (wl, layer)
+    if key not in _cache:
+        _cache.clear()
+        w = awq_synth.WORKLOADS[wl]
+        L = w.layer(layer)
+        W = awq_synth.layer_weight(0, w, L)
+        dev = gpu_pack(W)
+        _cache[key] = (L, dev, packed_to_host(*dev))
+    return _cache[key]
+
+
+@pytest.mark.parametrize("wl,layer,M", DECODE_CASES)
+def test_decode_full_size(wl, layer, M):
+    L, dev, hp = _full_layer(wl, layer)
+    x = awq_synth.layer_input(0, awq_synth.WORKLOADS[wl], L, M)
+    y = _run(awq.awq_linear, x, dev, L.N)
+    rows = sample_rows(L.N, 96, seed=M)
+    y_ref, b = oracle_rows(x, *hp, L.N, L.K, rows)
+    check_close(y[:, rows], y_ref, b, f"{wl}/{layer} M={M}")
+
+
+PREFILL_CASES = [(l.name, M) for l in awq_synth.WORKLOADS["prefill"].layers for M in (512, 2048, 8192)]
+
+
+@pytest.mark.parametrize("layer,M", PREFILL_CASES)
+def test_prefill_full_size(layer, M):
+    """4096 random outputs, the first and last output tile, one full row and
+    one full column, against the oracle computed one by one."""
+    L, dev, hp = _full_layer("prefill", layer)
+    x = awq_synth.layer_input(0, awq_synth.WORKLOADS["prefill"], L, M)
+    y = _run(awq.awq_linear, x, dev, L.N)
+    rng = np.random.default_rng(M)
+    ms = [rng.integers(0, M, 4096)]
+    ns = [rng.integers(0, L.N, 4096)]
+    for m0, n0 in ((0, 0), (M - 1, L.N - 1)):        # first / last 128 x 128 corner tiles, 8x8 subsampled
+        mm = np.arange(max(0, m0 - 127), min(M, m0 + 128))[::16]
+        nn = np.arange(max(0, n0 - 127), min(L.N, n0 + 128))[::16]
+        ms.append(np.repeat(mm, len(nn)))
+        ns.append(np.tile(nn, len(mm)))
+    mr = rng.integers(0, M)
+    ms.append(np.full(L.N, mr)), ns.append(np.arange(L.N))                 # a full row of y
+    nc = rng.integers(0, L.N)
+    ms.append(np.arange(M)), ns.append(np.full(M, nc))                     # a full column of y
+    ms, ns = np.concatenate(ms), np.concatenate(ns)
+    order = np.argsort(ns, kind="stable")
+    y_ref, b = oracle.linear_entries(x, *hp, L.N, L.K, ms[order], ns[order])
+    check_close(y[ms[order], ns[order]], y_ref, b, f"prefill/{layer} M={M}")

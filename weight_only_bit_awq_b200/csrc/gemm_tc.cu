@@ -1,0 +1,377 @@
+// Context-stage (prefill) W4A16 GEMM on the sm_100a tensor cores
+// (awq_w4a16_gemm).
+//
+// TinyChat README, "New Optimization of Context Stage": the prompt's tokens
+// go through the same 4-bit linear layers as one batch, so for M in the
+// hundreds to thousands the layer is a dense contraction and belongs on the
+// tensor cores. The weights are dequantized just ahead of the MMA.
+//
+// Tile: 128 output channels (the MMA M dimension, "swap AB": the weight is
+// operand A) x BN tokens (operand B, BN = 128 or 256) x the whole K, one tile
+// per CTA. Accumulation in tensor memory (fp32, BN columns x 128 lanes).
+//
+// Warp roles (224 threads):
+//   warp 0  lane 0 issues TMA loads of x: 64-k x BN boxes with the 128-byte
+//           swizzle, exactly the K-major operand layout tcgen05 reads.
+//   warp 1  allocates tensor memory; lane 0 issues tcgen05.mma (4 per 64-k
+//           stage, K = 16 each) and commits to the stage barriers.
+//   warp 2  lane 0 issues TMA loads of the packed weight: one 8 KiB box per
+//           128-k block (8 row blocks of 1 KiB).
+//   warps 3-6 dequantize: thread r owns weight row r of the tile, reads its
+//           64 B of codes for the k-block from shared memory, forms
+//           fp16_rne((q - z) * s) (the exact value the dequant kernel and the
+//           CPU oracle produce) and stores it, swizzled, into the A-operand
+//           buffer; afterwards they drain the accumulator (tcgen05.ld) and
+//           write fp16 y.
+// Rings: x 4 x (BN x 64 k), dequantized weight 2 x (128 x 128 k), packed
+// weight 3 x 8 KiB, each with full/empty mbarriers. Every wait is bounded
+// (2 s of %globaltimer); on expiry the CTA records AWQ_ERR_TIMEOUT in the
+// status word, the other roles stop at their next wait, in-flight copies and
+// MMAs are drained, tensor memory is freed and the CTA exits.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "awq_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace awq {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kXStages = 4;
+constexpr int kWStages = 2;
+constexpr int kQStages = 3;
+constexpr int kQBytes = 8 * 1024;
+constexpr int kWHalfBytes = kBM * 64 * 2;  // 16 KiB: 128 rows x 64 k
+constexpr int kWBytes = 2 * kWHalfBytes;
+constexpr int kWarpX = 0, kWarpMma = 1, kWarpQ = 2, kFirstDeqWarp = 3, kNumDeqWarps = 4;
+constexpr int kDeqThreads = kNumDeqWarps * 32;
+constexpr int kThreads = (kFirstDeqWarp + kNumDeqWarps) * 32;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kDrainLimitNs = 200000000ull;
+
+// barrier indices
+constexpr int kBarXFull = 0, kBarXEmpty = kBarXFull + kXStages, kBarWFull = kBarXEmpty + kXStages,
+              kBarWEmpty = kBarWFull + kWStages, kBarQFull = kBarWEmpty + kWStages,
+              kBarQEmpty = kBarQFull + kQStages, kBarAcc = kBarQEmpty + kQStages, kBarDrain = kBarAcc + 1,
+              kNumBars = kBarDrain + 1;
+
+template <int BN>
+struct Layout {
+  static constexpr int kXBytes = BN * 64 * 2;
+  static constexpr int kXOff = 0;
+  static constexpr int kWOff = kXOff + kXStages * kXBytes;
+  static constexpr int kQOff = kWOff + kWStages * kWBytes;
+  static constexpr int kBarOff = kQOff + kQStages * kQBytes;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1 KiB
+};
+static_assert(Layout<256>::kAlloc <= 232448, "shared memory budget");
+
+// Bounded wait on an mbarrier phase. Returns false when this CTA is aborting
+// (another role gave up) or when the wait itself ran past kWaitLimitNs (then
+// it records the timeout and starts the abort).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                         uint32_t* status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1; it < (1u << 30); ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (*abort_flag) return false;
+      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
+  }
+  *abort_flag = 1;
+  record_status(status, AWQ_ERR_TIMEOUT);
+  return false;
+}
+
+// Wait used only while aborting: for copies / MMAs already issued to land.
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 0; it < (1u << 30); ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return;
+    if ((it & 63) == 0 && ptx::globaltimer_ns() - t0 > kDrainLimitNs) return;
+  }
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// Eight codes of one word (k = 8w .. 8w+7) -> eight fp16 W^ = fp16_rne((q - z) s).
+// (word & 0x000F000F) | 0x64006400 = half2(1024 + q_even, 1024 + q_odd); the
+// 0x00F000F0 mask gives 1024 + 16 q. Subtracting 1024 + z (or scaling by 1/16
+// and subtracting 64 + z) is exact, and so the only rounding is that of the
+// final product by s (one IEEE fp16 multiply).
+__device__ __forceinline__ uint4 dequant_word(uint32_t w, __half2 zlo, __half2 zhi, __half2 s2) {
+  const __half2 sixteenth = __half2half2(__ushort_as_half(0x2C00));  // 1/16
+  uint4 o;
+  o.x = h2u(__hmul2(__hsub2(u2h(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), zlo), s2));
+  o.y = h2u(__hmul2(__hfma2(u2h(lop3_and_or(w, 0x00F000F0u, 0x64006400u)), sixteenth, zhi), s2));
+  w >>= 8;
+  o.z = h2u(__hmul2(__hsub2(u2h(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), zlo), s2));
+  o.w = h2u(__hmul2(__hfma2(u2h(lop3_and_or(w, 0x00F000F0u, 0x64006400u)), sixteenth, zhi), s2));
+  return o;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
+                const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M,
+                int K, int N, uint32_t* status) {
+  using L = Layout<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBarOff + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * BN;
+  const int n0 = blockIdx.y * kBM;
+  const int KB = K / kKPerBlock;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kXStages; ++i) {
+      ptx::mbar_init(bar(kBarXFull + i), 1);
+      ptx::mbar_init(bar(kBarXEmpty + i), 1);
+    }
+    for (int i = 0; i < kWStages; ++i) {
+      ptx::mbar_init(bar(kBarWFull + i), kDeqThreads);
+      ptx::mbar_init(bar(kBarWEmpty + i), 1);
+    }
+    for (int i = 0; i < kQStages; ++i) {
+      ptx::mbar_init(bar(kBarQFull + i), 1);
+      ptx::mbar_init(bar(kBarQEmpty + i), kDeqThreads);
+    }
+    ptx::mbar_init(bar(kBarAcc), 1);
+    ptx::mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == kWarpX && lane == 0) {
+    ptx::prefetch_tensormap(&tmap_x);
+    ptx::prefetch_tensormap(&tmap_q);
+  }
+  if (warp == kWarpMma) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), BN);
+    ptx::tmem_relinquish();
+    ptx::tc_fence_before();
+  }
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == kWarpX) {
+    // ---------------- x producer ----------------
+    if (lane == 0) {
+      const int nst = 2 * KB;
+      int i = 0;
+      for (; i < nst; ++i) {
+        const int s = i % kXStages;
+        if (!wait_bar(bar(kBarXEmpty + s), ((i / kXStages) & 1) ^ 1, abort_flag, status)) break;
+        ptx::mbar_arrive_expect_tx(bar(kBarXFull + s), L::kXBytes);
+        ptx::tma_load_2d(sbase + L::kXOff + s * L::kXBytes, &tmap_x, i * 64, m0, bar(kBarXFull + s));
+      }
+      if (i < nst)  // aborting: let the copies already issued land
+        for (int j = (i > kXStages ? i - kXStages : 0); j < i; ++j)
+          drain_bar(bar(kBarXFull + j % kXStages), (j / kXStages) & 1);
+    }
+    __syncwarp();
+  } else if (warp == kWarpQ) {
+    // ---------------- packed-weight producer ----------------
+    if (lane == 0) {
+      int kb = 0;
+      for (; kb < KB; ++kb) {
+        const int s = kb % kQStages;
+        if (!wait_bar(bar(kBarQEmpty + s), ((kb / kQStages) & 1) ^ 1, abort_flag, status)) break;
+        ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), kQBytes);
+        ptx::tma_load_2d(sbase + L::kQOff + s * kQBytes, &tmap_q, kb * kWordsPerBlock, n0 / kRowsPerBlock,
+                         bar(kBarQFull + s));
+      }
+      if (kb < KB)
+        for (int j = (kb > kQStages ? kb - kQStages : 0); j < kb; ++j)
+          drain_bar(bar(kBarQFull + j % kQStages), (j / kQStages) & 1);
+    }
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = ptx::idesc_f16_f32(kBM, BN);
+      bool ok = true;
+      for (int kb = 0; kb < KB && ok; ++kb) {
+        const int ws = kb % kWStages;
+        if (!(ok = wait_bar(bar(kBarWFull + ws), (kb / kWStages) & 1, abort_flag, status))) break;
+        ptx::tc_fence_after();
+        for (int h = 0; h < 2; ++h) {
+          const int i = 2 * kb + h, s = i % kXStages;
+          if (!(ok = wait_bar(bar(kBarXFull + s), (i / kXStages) & 1, abort_flag, status))) break;
+          ptx::tc_fence_after();
+          const uint32_t a_base = sbase + L::kWOff + ws * kWBytes + h * kWHalfBytes;
+          const uint32_t b_base = sbase + L::kXOff + s * L::kXBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_f16_ss(tmem_base, ptx::desc_kmajor_sw128(a_base + 32 * kk),
+                            ptx::desc_kmajor_sw128(b_base + 32 * kk), idesc, (kb | h | kk) != 0);
+          ptx::mma_commit(bar(kBarXEmpty + s));
+        }
+        if (ok) ptx::mma_commit(bar(kBarWEmpty + ws));
+      }
+      if (ok) {
+        ptx::mma_commit(bar(kBarAcc));
+      } else {  // aborting: wait for the MMAs already issued
+        ptx::mma_commit(bar(kBarDrain));
+        drain_bar(bar(kBarDrain), 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- dequantize, then epilogue ----------------
+    const int row = threadIdx.x - kFirstDeqWarp * 32;  // 0..127, row & 31 == lane
+    const int n = n0 + row;
+    const bool valid = n < N;
+    const int rot = (lane >> 1) & 3;  // chunk rotation: conflict-free shared loads and stores
+    bool ok = true;
+    float s_next = 0.f;
+    uint32_t z_next = 0;
+    if (valid) {
+      s_next = __half2float(scales[n]);
+      z_next = (zeros[n >> 1] >> (4 * (n & 1))) & 0xF;
+    }
+    for (int kb = 0; kb < KB; ++kb) {
+      const float s = s_next;
+      const uint32_t z = z_next;
+      if (valid && kb + 1 < KB) {
+        s_next = __half2float(scales[(int64_t)(kb + 1) * N + n]);
+        z_next = (zeros[(int64_t)(kb + 1) * (N / 2) + (n >> 1)] >> (4 * (n & 1))) & 0xF;
+      }
+      const int qs = kb % kQStages;
+      if (!(ok = wait_bar(bar(kBarQFull + qs), (kb / kQStages) & 1, abort_flag, status))) break;
+      const uint8_t* qrow = smem + L::kQOff + qs * kQBytes + (row >> 4) * 1024 + (row & 15) * 64;
+      uint4 c[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 3));
+      ptx::mbar_arrive(bar(kBarQEmpty + qs));
+
+      const int ws = kb % kWStages;
+      if (!(ok = wait_bar(bar(kBarWEmpty + ws), ((kb / kWStages) & 1) ^ 1, abort_flag, status))) break;
+      const __half2 s2 = __half2half2(__float2half_rn(s));
+      const __half2 zlo = __half2half2(__ushort_as_half((unsigned short)(0x6400u + z)));
+      const __half2 zhi = __half2half2(__float2half_rn(-64.0f - (float)z));
+      uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int cj = (jj + rot) & 3;  // which 32-k chunk of the block c[jj] holds
+        uint8_t* dst = wt + (cj >> 1) * kWHalfBytes;
+        const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
+#pragma unroll
+        for (int ww = 0; ww < 4; ++ww) {
+          const int chunk = 4 * (cj & 1) + ww;  // 16-byte chunk (8 k) within the 64-k half
+          *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) = dequant_word(words[ww], zlo, zhi, s2);
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(bar(kBarWFull + ws));
+    }
+    if (ok && wait_bar(bar(kBarAcc), 0, abort_flag, status)) {
+      ptx::tc_fence_after();
+      const int quad = warp & 3;  // this warp may read TMEM lanes 32*quad .. +31
+      const int r = 32 * quad + lane;
+      const int nn = n0 + r;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        if (m0 + c0 >= M) break;
+        uint32_t v[32];
+        ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)c0, v);
+        ptx::tmem_wait_ld();
+        if (nn < N) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int m = m0 + c0 + j;
+            if (m < M) y[(int64_t)m * N + nn] = __float2half_rn(__uint_as_float(v[j]));
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, BN);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+template <int BN>
+cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
+                      __half* y, int64_t M, int64_t K, int64_t N, uint32_t* status, cudaStream_t stream) {
+  using L = Layout<BN>;
+  auto encode = get_encode();
+  if (!encode) return cudaErrorNotSupported;
+  CUtensorMap tx, tq;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)BN};
+    cuuint32_t estr[2] = {1, 1};
+    if (encode(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const int64_t KB = K / kKPerBlock;
+    cuuint64_t dims[2] = {(cuuint64_t)(KB * kWordsPerBlock), (cuuint64_t)(N / kRowsPerBlock)};
+    cuuint64_t strides[1] = {(cuuint64_t)(KB * kWordsPerBlock * 4)};
+    cuuint32_t box[2] = {(cuuint32_t)kWordsPerBlock, (cuuint32_t)(kBM / kRowsPerBlock)};
+    cuuint32_t estr[2] = {1, 1};
+    if (encode(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qweight), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  static uint64_t attr_set = 0;  // one bit per device that has the attribute
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
+  if (!(attr_set >> dev & 1)) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set |= uint64_t(1) << dev;
+  }
+  dim3 grid((unsigned)((M + BN - 1) / BN), (unsigned)((N + kBM - 1) / kBM));
+  gemm_kernel<BN><<<grid, kThreads, L::kAlloc, stream>>>(tx, tq, scales, zeros, y, (int)M, (int)K, (int)N, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
+                        __half* y, int64_t M, int64_t K, int64_t N, uint32_t* status, cudaStream_t stream) {
+  if (M > 128) return launch_bn<256>(x, qweight, scales, zeros, y, M, K, N, status, stream);
+  return launch_bn<128>(x, qweight, scales, zeros, y, M, K, N, status, stream);
+}
+
+}  // namespace awq
