@@ -407,6 +407,46 @@ def run_ours(args):
     return 0
 
 
+SINGLE = {
+    # one kernel on a layer larger than the 126 MB L2, for profiler captures
+    "gemv": ("llama2_70b_decode", "gate_up", 1),     # 235 MB packed weight, M = 1
+    "gemm": ("prefill", "llama3_gate_up", 2048),     # 58 MB weight + 16 MB x + 117 MB y
+}
+
+
+def run_single(args):
+    """Launch one kernel `--reps` times on one full-size layer (no graphs),
+    then check the status word. Used as the target of ncu captures."""
+    import torch
+
+    import weight_only_bit_awq_b200 as awq
+    wl_name, layer_name, M = SINGLE[args.single]
+    wl = awq_synth.WORKLOADS[wl_name]
+    L = wl.layer(layer_name)
+    dev = torch.device("cuda", 0)
+    W = torch.from_numpy(awq_synth.layer_weight(0, wl, L).view(np.uint16)).view(torch.float16).to(dev)
+    ws = awq.new_workspace(M, L.K, L.N, dev)
+    packed = awq.awq_pack(W, ws)
+    del W
+    x = torch.from_numpy(awq_synth.layer_input(0, wl, L, M).view(np.uint16)).view(torch.float16).to(dev)
+    y = torch.empty((M, L.N), dtype=torch.float16, device=dev)
+    fn = awq.awq_w4a16_gemv if args.single == "gemv" else awq.awq_w4a16_gemm
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.reps + 1)]
+    ev[0].record()
+    for i in range(args.reps):
+        fn(x, *packed, L.N, ws, y=y)
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    st = awq.awq_get_status(ws)
+    if st != awq.AWQ_OK:
+        raise RuntimeError(awq.awq_status_string(st))
+    times = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.reps)]
+    work = (algo_bytes(M, L.K, L.N) / 1e9, "GB") if args.single == "gemv" else (2.0 * M * L.N * L.K / 1e12, "TFLOP")
+    print(json.dumps({"single": args.single, "workload": f"{wl_name}/{layer_name} K={L.K} N={L.N} M={M}",
+                      "ms": times, "rate_per_s": [work[0] / (t * 1e-3) for t in times], "unit": work[1] + "/s"}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -417,11 +457,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-frac", type=float, default=1.0, help="share of rows in the CPU-baseline sample")
     ap.add_argument("--ref-budget", type=float, default=60.0, help="seconds of oracle work in the reference arm")
+    ap.add_argument("--single", choices=sorted(SINGLE), help="launch one kernel on one layer (profiling target)")
+    ap.add_argument("--reps", type=int, default=4)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.single:
+        return run_single(args)
     return run_ours(args)
 
 

@@ -47,10 +47,19 @@ class _PackedSizes(ctypes.Structure):
                 ("zeros_bytes", ctypes.c_size_t)]
 
 
+def _build_module():
+    """build.py loaded by path (importing it must not load the library)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_awq_b200_build", os.path.join(_PKG, "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
 def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        from . import build as _build   # compile in-tree (nvcc); raises if that fails
-        _build.build()
+    # (Re)compile in-tree with nvcc when the library is missing or older than
+    # its sources; a failed build raises, there is no fallback.
+    _build_module().build()
     lib = ctypes.CDLL(LIB_PATH)
     vp, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     lib.awq_packed_size.argtypes = [i64, i64, ci, ctypes.POINTER(_PackedSizes)]

@@ -1,6 +1,6 @@
 """Build libawq_b200.so in-tree with nvcc for sm_100a.
 
-Usage: python -m weight_only_bit_awq_b200.build [--force] [--verbose]
+Usage: python weight_only_bit_awq_b200/build.py [--force] [--verbose]
 """
 from __future__ import annotations
 
