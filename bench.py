@@ -49,6 +49,22 @@ def algo_bytes(M, K, N, group=128):
     return K * N // 2 + 2 * (K // group) * N + (K // group) * N // 2 + 2 * M * K + 2 * M * N
 
 
+def reduce_max(v: float, world: int, device=None) -> float:
+    """Max of a per-rank value over all ranks (the process group's backend)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate_gbs(bytes_per_step: float, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job GB/s: the bytes every rank moved over the slowest rank's time."""
+    return bytes_per_step * steps * world / (ms_max * 1e-3) / 1e9
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -233,11 +249,7 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, world, dev)
 
     hbm, tc_burst, tc_sus, peak_kind = peaks()
     wl = awq_synth.WORKLOADS[WORKLOAD]
@@ -304,8 +316,8 @@ def run_ours(args):
     st = awq.awq_get_status(ws)
     if st != awq.AWQ_OK:
         raise RuntimeError(awq.awq_status_string(st))
-    value = step_bytes * args.steps * world / (ms * 1e-3) / 1e9
-    per_gpu_gbs = step_bytes * args.steps / (ms * 1e-3) / 1e9
+    value = job_rate_gbs(step_bytes, args.steps, world, ms)
+    per_gpu_gbs = job_rate_gbs(step_bytes, args.steps, 1, ms)
 
     # ---- end to end through the public API with pinned host buffers ----
     xh = [torch.empty_like(x, device="cpu").pin_memory().copy_(x.cpu()) for x in xs]
@@ -330,7 +342,7 @@ def run_ours(args):
         e1.record(stream)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e = {"value": step_bytes * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+    e2e = {"value": job_rate_gbs(step_bytes, e2e_steps, world, e2e_ms), "unit": "GB/s",
            "h2d_bytes_per_step": sum(x.numel() * 2 for x in xs),
            "d2h_bytes_per_step": sum(y.numel() * 2 for y in ys),
            "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
