@@ -142,6 +142,28 @@ awq_status awq_linear(const void* x, const void* qweight, const void* scales, co
 /* The M at and below which awq_linear takes the GEMV path. */
 int awq_linear_gemv_limit(void);
 
+/* Size of the library-owned scratch array behind awq_w4a16_gemv_no_alloc:
+ * 1 MiB of device memory on every GPU that loads the library, held until the
+ * process exits. */
+#define AWQ_GEMV_NO_ALLOC_SCRATCH_BYTES (1u << 20)
+
+/* The decode GEMV (awq_w4a16_gemv, same result bit for bit) for callers that
+ * cannot allocate device memory -- e.g. code running inside a fixed memory
+ * pool it must not grow, or a plug-in whose host process owns every device
+ * allocation. The pages have no counterpart of this entry point. Same
+ * arguments as awq_w4a16_gemv minus the workspace: the split-K scratch lives
+ * in a static device array of AWQ_GEMV_NO_ALLOC_SCRATCH_BYTES inside the
+ * library, so nothing is allocated (no cudaMalloc, no allocating library
+ * call). Returns AWQ_ERR_WORKSPACE when these sizes need more scratch than
+ * that (awq_workspace_bytes(M, K, N, group) > AWQ_GEMV_NO_ALLOC_SCRATCH_BYTES).
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. Every call uses the same array: calls that can
+ * overlap on the GPU race on it. Each call zeroes the counters it needs
+ * (a memset on `stream`) before its kernel runs. */
+awq_status awq_w4a16_gemv_no_alloc(const void* x, const void* qweight, const void* scales, const void* zeros,
+                                   void* y, int64_t M, int64_t K, int64_t N, int group, void* stream);
+
 /* Synchronize `stream`, then return and clear the device-side status word of
  * `workspace` (AWQ_OK if no device-side error was recorded). */
 awq_status awq_get_status(void* workspace, void* stream);

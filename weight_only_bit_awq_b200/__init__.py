@@ -9,7 +9,8 @@ importing the binding fails loudly if the shared library cannot be loaded.
 Functions (same names as the C entry points):
   awq_packed_size, awq_workspace_bytes, awq_workspace_init, awq_pack,
   awq_dequant, awq_w4a16_gemv, awq_w4a16_gemm, awq_linear,
-  awq_linear_gemv_limit, awq_get_status, awq_status_string.
+  awq_linear_gemv_limit, awq_get_status, awq_status_string,
+  awq_w4a16_gemv_no_alloc.
 """
 from __future__ import annotations
 
@@ -33,7 +34,7 @@ globals().update({name: code for code, name in STATUS_NAMES.items()})
 # Every symbol include/awq.h declares.
 EXPORTS = ("awq_packed_size", "awq_workspace_bytes", "awq_workspace_init", "awq_pack", "awq_dequant",
            "awq_w4a16_gemv", "awq_w4a16_gemm", "awq_linear", "awq_linear_gemv_limit", "awq_get_status",
-           "awq_status_string")
+           "awq_status_string", "awq_w4a16_gemv_no_alloc")
 
 
 class AwqError(RuntimeError):
@@ -70,6 +71,7 @@ def _load() -> ctypes.CDLL:
     lib.awq_dequant.argtypes = [vp, vp, vp, i64, i64, ci, vp, vp]
     for f in ("awq_w4a16_gemv", "awq_w4a16_gemm", "awq_linear"):
         getattr(lib, f).argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, sz, vp]
+    lib.awq_w4a16_gemv_no_alloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp]
     lib.awq_linear_gemv_limit.argtypes = []
     lib.awq_get_status.argtypes = [vp, vp]
     lib.awq_status_string.argtypes = [ci]
@@ -178,6 +180,20 @@ def awq_w4a16_gemm(x, qweight, scales, zeros, N, workspace, group: int = GROUP, 
 def awq_linear(x, qweight, scales, zeros, N, workspace, group: int = GROUP, y=None):
     """The linear layer: GEMV for M <= awq_linear_gemv_limit(), GEMM above."""
     return _linear_call(lib.awq_linear, "awq_linear", x, qweight, scales, zeros, N, workspace, group, y)
+
+
+def awq_w4a16_gemv_no_alloc(x, qweight, scales, zeros, N, group: int = GROUP, y=None):
+    """Decode GEMV for callers that cannot allocate device memory: no
+    workspace argument; the library's own static scratch array is used (see
+    include/awq.h). Here torch allocates y only when the caller passes none."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _check(lib.awq_w4a16_gemv_no_alloc(_dev(x, torch.float16, "x"), _dev(qweight, torch.int32, "qweight"),
+                                       _dev(scales, torch.float16, "scales"), _dev(zeros, torch.uint8, "zeros"),
+                                       _dev(y, torch.float16, "y"), M, K, N, group, _stream(x)),
+           "awq_w4a16_gemv_no_alloc")
+    return y
 
 
 def awq_linear_gemv_limit() -> int:
