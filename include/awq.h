@@ -17,14 +17,18 @@
  * ---------------------------------------------------------------------------
  * Packed layout (ours; the README names only a "-w4-g128-awq.pt" checkpoint)
  * ---------------------------------------------------------------------------
- *   qweight  uint32 [N/16][K/128][16][16]   (K*N/2 bytes)
+ *   qweight  uint32, (N/16)*(K/128) blocks of 16 x 16 words (K*N/2 bytes)
  *            Block (nb, kb) is 1 KiB, holds output channels n = 16*nb + r
  *            (r = 0..15) and input channels 128*kb .. 128*kb + 127. Word w of
  *            row r holds k = 128*kb + 8*w + i for i = 0..7: the code of even i
  *            at bits 4*(i/2) .. 4*(i/2)+3 and the code of odd i at bits
  *            16 + 4*(i/2) .. 16 + 4*(i/2)+3. So (word >> 4*j) & 0x000F000F
  *            holds the adjacent pair k = 8w + 2j, 8w + 2j + 1 as two 16-bit
- *            lanes, and a 16x128 tile is one contiguous 1 KiB load.
+ *            lanes. Blocks are grouped by 8 row blocks (128 output channels):
+ *            group gi = nb/8 holds R = min(8, N/16 - 8*gi) row blocks and is
+ *            stored k-block-major, so block (nb, kb) is block number
+ *            8*gi*(K/128) + kb*R + nb%8, and the R blocks of one k-block of
+ *            one group (128 x 128 weights) are one contiguous run of R KiB.
  *   scales   fp16  [K/group][N]             (2*N*K/group bytes)
  *   zeros    uint8 [K/group][N/2]           (N*K/(2*group) bytes): the zero
  *            point of even n in the low nibble, of odd n in the high nibble.
@@ -57,9 +61,10 @@
  *              awq_get_status.
  *   Workspace  at least awq_workspace_bytes(M, K, N, group) bytes of device
  *              memory, zeroed once with awq_workspace_init before first use.
- *              Kernels leave it zeroed again (split-K counters reset
- *              themselves). One workspace must not be used by two calls that
- *              can run at the same time (e.g. on two streams).
+ *              Only its status word must start at zero; the GEMV's partial
+ *              sums of split rows are written before they are read. One
+ *              workspace must not be used by two calls that can run at the
+ *              same time (e.g. on two streams).
  */
 #ifndef AWQ_B200_H
 #define AWQ_B200_H
@@ -97,7 +102,7 @@ typedef struct awq_packed_sizes {
 awq_status awq_packed_size(int64_t K, int64_t N, int group, awq_packed_sizes* out);
 
 /* Workspace bytes needed by any entry point below for these sizes on the
- * current device (split-K partials, counters, the status word). Host only.
+ * current device (the status word, the GEMV's partial sums of rows split between CTAs). Host only.
  * Returns 0 for invalid sizes. */
 size_t awq_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
 
@@ -151,7 +156,7 @@ int awq_linear_gemv_limit(void);
  * cannot allocate device memory -- e.g. code running inside a fixed memory
  * pool it must not grow, or a plug-in whose host process owns every device
  * allocation. The pages have no counterpart of this entry point. Same
- * arguments as awq_w4a16_gemv minus the workspace: the split-K scratch lives
+ * arguments as awq_w4a16_gemv minus the workspace: the workspace lives
  * in a static device array of AWQ_GEMV_NO_ALLOC_SCRATCH_BYTES inside the
  * library, so nothing is allocated (no cudaMalloc, no allocating library
  * call). Returns AWQ_ERR_WORKSPACE when these sizes need more scratch than
@@ -159,10 +164,24 @@ int awq_linear_gemv_limit(void);
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture. Every call uses the same array: calls that can
- * overlap on the GPU race on it. Each call zeroes the counters it needs
- * (a memset on `stream`) before its kernel runs. */
+ * overlap on the GPU race on it. Each call zeroes the status word (a memset
+ * on `stream`) before its kernels run. */
 awq_status awq_w4a16_gemv_no_alloc(const void* x, const void* qweight, const void* scales, const void* zeros,
                                    void* y, int64_t M, int64_t K, int64_t N, int group, void* stream);
+
+/* Number of kernels awq_linear launches for these sizes on the current device
+ * (1, or 2 when the decode GEMV also runs its split-row fixup kernel; 0 for
+ * M == 0 or invalid sizes). Host only. For launch accounting and graph planning;
+ * the pages have no counterpart. */
+int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group);
+
+/* Self-test of the kernels' failure detection (the pages have no counterpart):
+ * launches one thread that waits, through the same bounded-wait routine the
+ * GEMM and GEMV pipelines use, on a barrier phase that nothing completes,
+ * giving up after `limit_us` microseconds (1 .. 1000000). The expired wait
+ * records AWQ_ERR_TIMEOUT in the workspace status word, which awq_get_status
+ * then returns; the CUDA context stays usable. Returns AWQ_OK when launched. */
+awq_status awq_check_bounded_wait(void* workspace, size_t ws_bytes, uint32_t limit_us, void* stream);
 
 /* Synchronize `stream`, then return and clear the device-side status word of
  * `workspace` (AWQ_OK if no device-side error was recorded). */

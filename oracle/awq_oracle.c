@@ -26,12 +26,18 @@
  *   - a second, independent matmul route that factors the zero point out of
  *     each group:  y[m,n] = sum_g s * (sum_{k in g} x*q  -  z * sum_{k in g} x).
  *   - the packed layout (our own; the pages only name a ".pt" checkpoint):
- *       qweight  uint32 [N/16][K/128][16][16]: block (nb, kb) holds rows
- *                n = 16nb + r (r = 0..15) and input channels 128kb..128kb+127;
- *                word w of row r holds k = 128kb + 8w + i, i = 0..7, with the
- *                nibble of even i at bits 4*(i/2) and of odd i at bits
- *                16 + 4*(i/2).  (So (word >> 4j) & 0x000F000F holds the
- *                adjacent pair k = 8w+2j, 8w+2j+1 as two 16-bit lanes.)
+ *       qweight  uint32, 1 KiB blocks of 16 rows x 128 input channels.
+ *                Block (nb, kb) holds rows n = 16nb + r (r = 0..15) and
+ *                k = 128kb .. 128kb+127; word w of row r holds
+ *                k = 128kb + 8w + i, i = 0..7, with the nibble of even i at
+ *                bits 4*(i/2) and of odd i at bits 16 + 4*(i/2).  (So
+ *                (word >> 4j) & 0x000F000F holds the adjacent pair
+ *                k = 8w+2j, 8w+2j+1 as two 16-bit lanes.)
+ *                Blocks are grouped by 8 row blocks (128 rows): group
+ *                gi = nb / 8 has R = min(8, N/16 - 8gi) row blocks and is
+ *                stored k-block-major, so block (nb, kb) is block number
+ *                8*gi*(K/128) + kb*R + nb%8 and the R blocks of one k-block of
+ *                one group are contiguous.
  *       scales   fp16  [K/G][N]
  *       zeros    uint8 [K/G][N/2]: low nibble = even n, high nibble = odd n.
  *
@@ -167,10 +173,14 @@ int orc_dequant(const uint8_t* q, const uint8_t* z, const uint16_t* s, int64_t N
 /* Bit position of element i (0..7) inside its 32-bit word. */
 static int nibble_shift(int i) { return (i % 2 == 0) ? 4 * (i / 2) : 16 + 4 * (i / 2); }
 
-/* Index of the word holding (n, k) in qweight [N/16][K/128][16][16]. */
-static int64_t word_index(int64_t n, int64_t k, int64_t K) {
+/* Index of the word holding (n, k): block number (group-major, k-block,
+ * row block within the group), then row r and word w inside the block. */
+static int64_t word_index(int64_t n, int64_t k, int64_t K, int64_t N) {
   int64_t nb = n / 16, r = n % 16, kb = k / 128, w = (k % 128) / 8;
-  return ((nb * (K / 128) + kb) * 16 + r) * 16 + w;
+  int64_t gi = nb / 8, NB = N / 16;
+  int64_t rows_in_group = (NB - 8 * gi < 8) ? NB - 8 * gi : 8;
+  int64_t block = 8 * gi * (K / 128) + kb * rows_in_group + nb % 8;
+  return (block * 16 + r) * 16 + w;
 }
 
 int orc_pack(const uint8_t* q, const uint8_t* z, const uint16_t* s, int64_t N, int64_t K, int G,
@@ -181,7 +191,7 @@ int orc_pack(const uint8_t* q, const uint8_t* z, const uint16_t* s, int64_t N, i
   memset(zeros, 0, (size_t)(ng * N / 2));
   for (int64_t n = 0; n < N; ++n)
     for (int64_t k = 0; k < K; ++k)
-      qweight[word_index(n, k, K)] |= (uint32_t)(q[n * K + k] & 0xF) << nibble_shift((int)(k % 8));
+      qweight[word_index(n, k, K, N)] |= (uint32_t)(q[n * K + k] & 0xF) << nibble_shift((int)(k % 8));
   for (int64_t g = 0; g < ng; ++g)
     for (int64_t n = 0; n < N; ++n) {
       scales[g * N + n] = s[n * ng + g];
@@ -196,7 +206,7 @@ int orc_unpack(const uint32_t* qweight, const uint16_t* scales, const uint8_t* z
   int64_t ng = K / G;
   for (int64_t n = 0; n < N; ++n)
     for (int64_t k = 0; k < K; ++k)
-      q[n * K + k] = (uint8_t)((qweight[word_index(n, k, K)] >> nibble_shift((int)(k % 8))) & 0xF);
+      q[n * K + k] = (uint8_t)((qweight[word_index(n, k, K, N)] >> nibble_shift((int)(k % 8))) & 0xF);
   for (int64_t g = 0; g < ng; ++g)
     for (int64_t n = 0; n < N; ++n) {
       s[n * ng + g] = scales[g * N + n];
@@ -262,7 +272,7 @@ static void packed_row(const uint32_t* qweight, const uint16_t* scales, const ui
                        int64_t K, int G, int64_t n, double* row) {
   for (int64_t k = 0; k < K; ++k) {
     int64_t g = k / G;
-    uint32_t q = (qweight[word_index(n, k, K)] >> nibble_shift((int)(k % 8))) & 0xF;
+    uint32_t q = (qweight[word_index(n, k, K, N)] >> nibble_shift((int)(k % 8))) & 0xF;
     uint32_t z = (zeros[g * (N / 2) + n / 2] >> (4 * (n % 2))) & 0xF;
     double s = orc_half_to_double(scales[g * N + n]);
     row[k] = orc_half_to_double(orc_double_to_half(((double)q - (double)z) * s));
