@@ -389,7 +389,7 @@ def run_ours(args):
                          f"({t:.1f} s, fp64 C oracle, single thread)"}
 
     traffic = traffic_per_launch()
-    launches = len(layers) * args.steps
+    launches = sum(awq.awq_linear_launches(M_DECODE, L.K, L.N) for L in layers) * args.steps
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",

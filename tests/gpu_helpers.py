@@ -42,6 +42,14 @@ def gpu_pack(W: np.ndarray, ws: torch.Tensor | None = None):
     return qw, sc, ze
 
 
+def block_of(nb: int, kb: int, KB: int, NB: int) -> int:
+    """Block number of row block nb, k-block kb in the packed layout of
+    include/awq.h (groups of 8 row blocks, k-block-major inside a group)."""
+    gi = nb // 8
+    R = min(8, NB - 8 * gi)
+    return 8 * gi * KB + kb * R + nb % 8
+
+
 def packed_to_host(qw, sc, ze):
     return host(qw, np.uint32), host(sc, np.float16), host(ze, np.uint8)
 

@@ -120,3 +120,18 @@ def test_valid_arguments_without_a_device_stop_at_the_device_check():
         assert _linear(fn) == awq.AWQ_ERR_UNSUPPORTED
     assert L.awq_pack(FAKE, 4096, 4096, 128, FAKE2, FAKE3, FAKE4, FAKE5, 1 << 20, None) == awq.AWQ_ERR_UNSUPPORTED
     assert L.awq_dequant(FAKE2, FAKE3, FAKE4, 4096, 4096, 128, FAKE, None) == awq.AWQ_ERR_UNSUPPORTED
+
+
+def test_linear_launch_counts():
+    assert awq.awq_linear_launches(0, 4096, 4096) == 0
+    assert awq.awq_linear_launches(1, 4000, 4096) == 0
+    assert awq.awq_linear_launches(2048, 4096, 4096) == 1          # the GEMM: one kernel
+    assert awq.awq_linear_launches(1, 4096, 4096) in (1, 2)        # the GEMV, plus its fixup when rows are split
+
+
+def test_bounded_wait_self_test_argument_errors():
+    assert L.awq_check_bounded_wait(None, 256, 1000, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_check_bounded_wait(FAKE, 256, 0, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_check_bounded_wait(FAKE, 256, 2000000, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_check_bounded_wait(FAKE + 4, 256, 1000, None) == awq.AWQ_ERR_ALIGNMENT
+    assert L.awq_check_bounded_wait(FAKE, 16, 1000, None) == awq.AWQ_ERR_WORKSPACE

@@ -6,7 +6,7 @@ import torch
 import awq_synth
 import oracle
 import weight_only_bit_awq_b200 as awq
-from gpu_helpers import gpu_pack, packed_to_host, to_dev, host
+from gpu_helpers import block_of, gpu_pack, host, packed_to_host, to_dev
 
 pytestmark = pytest.mark.gpu
 G = 128
@@ -111,6 +111,7 @@ def test_pack_bit_exact_full_size_sampled(wl, layer):
     for nb in blocks:
         rows = slice(16 * nb, 16 * nb + 16)
         oq, osc, oze = oracle.quantize_pack(np.ascontiguousarray(W[rows]))
-        assert (qw[nb] == oq.reshape(KB, 16, 16)).all(), nb
+        blocks_gpu = qw.reshape(-1, 16, 16)[[block_of(nb, kb, KB, L.N // 16) for kb in range(KB)]]
+        assert (blocks_gpu == oq.reshape(KB, 16, 16)).all(), nb
         assert (sc[:, rows].view(np.uint16) == osc.view(np.uint16)).all(), nb
         assert (ze[:, 8 * nb:8 * nb + 8] == oze).all(), nb

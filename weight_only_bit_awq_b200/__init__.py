@@ -9,8 +9,8 @@ importing the binding fails loudly if the shared library cannot be loaded.
 Functions (same names as the C entry points):
   awq_packed_size, awq_workspace_bytes, awq_workspace_init, awq_pack,
   awq_dequant, awq_w4a16_gemv, awq_w4a16_gemm, awq_linear,
-  awq_linear_gemv_limit, awq_get_status, awq_status_string,
-  awq_w4a16_gemv_no_alloc.
+  awq_linear_gemv_limit, awq_linear_launches, awq_check_bounded_wait,
+  awq_get_status, awq_status_string, awq_w4a16_gemv_no_alloc.
 """
 from __future__ import annotations
 
@@ -34,7 +34,7 @@ globals().update({name: code for code, name in STATUS_NAMES.items()})
 # Every symbol include/awq.h declares.
 EXPORTS = ("awq_packed_size", "awq_workspace_bytes", "awq_workspace_init", "awq_pack", "awq_dequant",
            "awq_w4a16_gemv", "awq_w4a16_gemm", "awq_linear", "awq_linear_gemv_limit", "awq_get_status",
-           "awq_status_string", "awq_w4a16_gemv_no_alloc")
+           "awq_status_string", "awq_w4a16_gemv_no_alloc", "awq_linear_launches", "awq_check_bounded_wait")
 
 
 class AwqError(RuntimeError):
@@ -73,6 +73,8 @@ def _load() -> ctypes.CDLL:
         getattr(lib, f).argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, sz, vp]
     lib.awq_w4a16_gemv_no_alloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp]
     lib.awq_linear_gemv_limit.argtypes = []
+    lib.awq_linear_launches.argtypes = [i64, i64, i64, ci]
+    lib.awq_check_bounded_wait.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.awq_get_status.argtypes = [vp, vp]
     lib.awq_status_string.argtypes = [ci]
     lib.awq_status_string.restype = ctypes.c_char_p
@@ -134,9 +136,10 @@ def new_workspace(M: int, K: int, N: int, device, group: int = GROUP) -> torch.T
 
 
 def awq_pack(w: torch.Tensor, workspace: torch.Tensor, group: int = GROUP):
-    """w fp16 [N][K] -> (qweight int32 [N/16][K/128][16][16], scales fp16 [K/G][N], zeros uint8 [K/G][N/2])."""
+    """w fp16 [N][K] -> (qweight int32 [(N/16)*(K/128)][16][16] packed blocks in the order
+    include/awq.h documents, scales fp16 [K/G][N], zeros uint8 [K/G][N/2])."""
     N, K = w.shape
-    qweight = torch.empty((N // 16, K // 128, 16, 16), dtype=torch.int32, device=w.device)
+    qweight = torch.empty(((N // 16) * (K // 128), 16, 16), dtype=torch.int32, device=w.device)
     scales = torch.empty((K // group, N), dtype=torch.float16, device=w.device)
     zeros = torch.empty((K // group, N // 2), dtype=torch.uint8, device=w.device)
     _check(lib.awq_pack(_dev(w, torch.float16, "w"), K, N, group, qweight.data_ptr(), scales.data_ptr(),
@@ -198,6 +201,18 @@ def awq_w4a16_gemv_no_alloc(x, qweight, scales, zeros, N, group: int = GROUP, y=
 
 def awq_linear_gemv_limit() -> int:
     return int(lib.awq_linear_gemv_limit())
+
+
+def awq_linear_launches(M: int, K: int, N: int, group: int = GROUP) -> int:
+    """Kernels awq_linear launches for these sizes on the current device."""
+    return int(lib.awq_linear_launches(M, K, N, group))
+
+
+def awq_check_bounded_wait(workspace: torch.Tensor, limit_us: int = 1000):
+    """Run the kernels' bounded wait on a barrier nothing completes (self-test);
+    afterwards awq_get_status(workspace) reports AWQ_ERR_TIMEOUT."""
+    _check(lib.awq_check_bounded_wait(_dev(workspace, torch.uint8, "workspace"), workspace.numel(), limit_us,
+                                      _stream(workspace)), "awq_check_bounded_wait")
 
 
 def awq_get_status(workspace: torch.Tensor) -> int:

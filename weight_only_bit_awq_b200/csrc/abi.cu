@@ -3,8 +3,24 @@
 #include <mutex>
 
 #include "awq_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace awq {
+
+namespace {
+// One thread waits, through the kernels' bounded-wait helper, on an mbarrier
+// phase that nothing will ever complete; the wait gives up after `limit_ns`
+// and records AWQ_ERR_TIMEOUT in the status word.
+__global__ void bounded_wait_probe_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t barrier;
+  __shared__ uint32_t abort_flag;
+  const uint32_t bar = ptx::smem_u32(&barrier);
+  ptx::mbar_init(bar, 1);
+  abort_flag = 0;
+  ptx::fence_mbarrier_init();
+  ptx::wait_bar(bar, 0, &abort_flag, status, limit_ns);
+}
+}  // namespace
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -224,6 +240,23 @@ awq_status awq_linear(const void* x, const void* qweight, const void* scales, co
 }
 
 int awq_linear_gemv_limit(void) { return g_gemv_limit; }
+
+int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group) {
+  if (M <= 0 || M > kMaxM || check_kn(K, N, group) != AWQ_OK) return 0;
+  if (M > g_gemv_limit) return 1;
+  return plan_gemv(M, K, N, sm_count_or_default()).has_split ? 2 : 1;
+}
+
+awq_status awq_check_bounded_wait(void* workspace, size_t ws_bytes, uint32_t limit_us, void* stream) {
+  if (!workspace || limit_us == 0 || limit_us > 1000000) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return AWQ_ERR_ALIGNMENT;
+  if (ws_bytes < kWsHeaderBytes) return AWQ_ERR_WORKSPACE;
+  awq_status st = check_device();
+  if (st != AWQ_OK) return st;
+  bounded_wait_probe_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(status_word(workspace),
+                                                                             (uint64_t)limit_us * 1000);
+  return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
 
 awq_status awq_get_status(void* workspace, void* stream) {
   if (!workspace) return AWQ_ERR_INVALID_ARG;

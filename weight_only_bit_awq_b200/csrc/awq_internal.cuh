@@ -16,10 +16,28 @@ constexpr int kKPerBlock = 128;
 constexpr int kWordsPerRow = kKPerBlock / 8;   // 16
 constexpr int kWordsPerBlock = kRowsPerBlock * kWordsPerRow;  // 256
 
+// Packed blocks are grouped by 8 row blocks (128 output channels); a group
+// holds R = min(8, NB - 8*gi) row blocks and is stored k-block-major, so the
+// R blocks of one (group, k-block) unit are one contiguous run of R KiB.
+constexpr int kGroupBlocks = 8;
+
+__host__ __device__ __forceinline__ int64_t group_rows(int64_t gi, int64_t NB) {
+  const int64_t r = NB - kGroupBlocks * gi;
+  return r < kGroupBlocks ? r : kGroupBlocks;
+}
+// First block of unit (gi, kb).
+__host__ __device__ __forceinline__ int64_t unit_first_block(int64_t gi, int64_t kb, int64_t KB, int64_t NB) {
+  return kGroupBlocks * gi * KB + kb * group_rows(gi, NB);
+}
+// Block number of row block nb, k-block kb.
+__host__ __device__ __forceinline__ int64_t block_index(int64_t nb, int64_t kb, int64_t KB, int64_t NB) {
+  return unit_first_block(nb / kGroupBlocks, kb, KB, NB) + nb % kGroupBlocks;
+}
+
 // Workspace layout (bytes):
 //   [0, 256)                   header: uint32 status word at offset 0
-//   [256, 256 + counters)      split-K arrival counters (uint32, rounded to 256 B)
-//   [.., + S*M*N*4)            split-K fp32 partial sums, slot-major [S][M][N]
+//   [partial_off, ws_bytes)    decode GEMV fp32 partial sums of row blocks split
+//                              between CTAs: [ctas][2][8][16][M]
 constexpr size_t kWsHeaderBytes = 256;
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -40,11 +58,13 @@ const DeviceInfo& device_info();   // current device
 
 // GEMV launch plan (shared by awq_workspace_bytes and the launcher).
 struct GemvPlan {
-  int nt;      // token tiles of 8 (1, 2 or 4)
-  int rb;      // row blocks (16 output channels each) per CTA
-  int splits;  // split-K factor
-  int ctas_n;  // CTAs along N = ceil(N/16 / rb)
-  size_t ws_bytes;
+  int nt;               // token tiles of 8 (1, 2 or 4)
+  int ctas;             // persistent CTAs (up to two per SM)
+  int groups;           // groups of 8 row blocks
+  bool has_split;       // some group is split between CTAs (the fixup kernel runs)
+  size_t partial_off;   // workspace offset of the split-row partial sums (bytes)
+  size_t zero_bytes;    // bytes at the start of the workspace that must be zero at launch
+  size_t ws_bytes;      // total workspace bytes
 };
 GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int sm_count);
 

@@ -15,8 +15,8 @@
 //           swizzle, exactly the K-major operand layout tcgen05 reads.
 //   warp 1  allocates tensor memory; lane 0 issues tcgen05.mma (4 per 64-k
 //           stage, K = 16 each) and commits to the stage barriers.
-//   warp 2  lane 0 issues TMA loads of the packed weight: one 8 KiB box per
-//           128-k block (8 row blocks of 1 KiB).
+//   warp 2  lane 0 issues bulk copies of the packed weight: the tile's 8 row
+//           blocks of one 128-k block are one contiguous 8 KiB run.
 //   warps 3-6 dequantize: thread r owns weight row r of the tile, reads its
 //           64 B of codes for the k-block from shared memory, forms
 //           fp16_rne((q - z) * s) (the exact value the dequant kernel and the
@@ -48,8 +48,6 @@ constexpr int kWBytes = 2 * kWHalfBytes;
 constexpr int kWarpX = 0, kWarpMma = 1, kWarpQ = 2, kFirstDeqWarp = 3, kNumDeqWarps = 4;
 constexpr int kDeqThreads = kNumDeqWarps * 32;
 constexpr int kThreads = (kFirstDeqWarp + kNumDeqWarps) * 32;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr uint64_t kDrainLimitNs = 200000000ull;
 
 // barrier indices
 constexpr int kBarXFull = 0, kBarXEmpty = kBarXFull + kXStages, kBarWFull = kBarXEmpty + kXStages,
@@ -70,33 +68,8 @@ struct Layout {
 };
 static_assert(Layout<256>::kAlloc <= 232448, "shared memory budget");
 
-// Bounded wait on an mbarrier phase. Returns false when this CTA is aborting
-// (another role gave up) or when the wait itself ran past kWaitLimitNs (then
-// it records the timeout and starts the abort).
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                         uint32_t* status) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = ptx::globaltimer_ns();
-  for (uint32_t it = 1; it < (1u << 30); ++it) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 0) {
-      if (*abort_flag) return false;
-      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) break;
-    }
-  }
-  *abort_flag = 1;
-  record_status(status, AWQ_ERR_TIMEOUT);
-  return false;
-}
-
-// Wait used only while aborting: for copies / MMAs already issued to land.
-__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = ptx::globaltimer_ns();
-  for (uint32_t it = 0; it < (1u << 30); ++it) {
-    if (ptx::mbar_try_wait(bar, parity)) return;
-    if ((it & 63) == 0 && ptx::globaltimer_ns() - t0 > kDrainLimitNs) return;
-  }
-}
+using ptx::drain_bar;
+using ptx::wait_bar;
 
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
@@ -124,7 +97,7 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, __half2 zlo, __half2 z
 
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
                 const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M,
                 int K, int N, uint32_t* status) {
   using L = Layout<BN>;
@@ -160,7 +133,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == kWarpX && lane == 0) {
     ptx::prefetch_tensormap(&tmap_x);
-    ptx::prefetch_tensormap(&tmap_q);
   }
   if (warp == kWarpMma) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), BN);
@@ -190,13 +162,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpQ) {
     // ---------------- packed-weight producer ----------------
     if (lane == 0) {
+      // The R <= 8 row blocks of this tile's group are one contiguous run of
+      // R KiB per k-block in the packed layout: one 1-D bulk copy each.
+      const int64_t NB = N / kRowsPerBlock, gi = blockIdx.y;
+      const uint32_t qbytes = (uint32_t)(group_rows(gi, NB) * 1024);
       int kb = 0;
       for (; kb < KB; ++kb) {
         const int s = kb % kQStages;
         if (!wait_bar(bar(kBarQEmpty + s), ((kb / kQStages) & 1) ^ 1, abort_flag, status)) break;
-        ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), kQBytes);
-        ptx::tma_load_2d(sbase + L::kQOff + s * kQBytes, &tmap_q, kb * kWordsPerBlock, n0 / kRowsPerBlock,
-                         bar(kBarQFull + s));
+        ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qbytes);
+        ptx::bulk_g2s(sbase + L::kQOff + s * kQBytes, qweight + unit_first_block(gi, kb, KB, NB) * kWordsPerBlock,
+                      qbytes, bar(kBarQFull + s));
       }
       if (kb < KB)
         for (int j = (kb > kQStages ? kb - kQStages : 0); j < kb; ++j)
@@ -331,7 +307,7 @@ cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* sc
   using L = Layout<BN>;
   auto encode = get_encode();
   if (!encode) return cudaErrorNotSupported;
-  CUtensorMap tx, tq;
+  CUtensorMap tx;
   {
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     cuuint64_t strides[1] = {(cuuint64_t)K * 2};
@@ -339,17 +315,6 @@ cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* sc
     cuuint32_t estr[2] = {1, 1};
     if (encode(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(x), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  {
-    const int64_t KB = K / kKPerBlock;
-    cuuint64_t dims[2] = {(cuuint64_t)(KB * kWordsPerBlock), (cuuint64_t)(N / kRowsPerBlock)};
-    cuuint64_t strides[1] = {(cuuint64_t)(KB * kWordsPerBlock * 4)};
-    cuuint32_t box[2] = {(cuuint32_t)kWordsPerBlock, (cuuint32_t)(kBM / kRowsPerBlock)};
-    cuuint32_t estr[2] = {1, 1};
-    if (encode(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qweight), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
@@ -362,7 +327,8 @@ cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* sc
     attr_set |= uint64_t(1) << dev;
   }
   dim3 grid((unsigned)((M + BN - 1) / BN), (unsigned)((N + kBM - 1) / kBM));
-  gemm_kernel<BN><<<grid, kThreads, L::kAlloc, stream>>>(tx, tq, scales, zeros, y, (int)M, (int)K, (int)N, status);
+  gemm_kernel<BN><<<grid, kThreads, L::kAlloc, stream>>>(tx, qweight, scales, zeros, y, (int)M, (int)K, (int)N,
+                                                          status);
   return cudaGetLastError();
 }
 

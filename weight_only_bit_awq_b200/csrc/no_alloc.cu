@@ -5,7 +5,8 @@
 // inside a custom memory pool it must not grow, plug-ins loaded into a host
 // process that owns all device allocations, or real-time paths where an
 // allocation may block on the driver. awq_w4a16_gemv needs a caller-provided
-// workspace for its split-K partial sums and arrival counters; this entry
+// workspace for its status word and the partial sums of rows split between
+// CTAs; this entry
 // point instead uses a fixed scratch array that lives in the library itself
 // (a file-scope __device__ array, one instance per GPU that loads the
 // library, held until the process exits), so the caller passes only its
@@ -17,7 +18,7 @@
 // that first call before any stream capture. Calls share the array: two
 // calls that can overlap on the GPU (different streams, or different host
 // threads on one stream without ordering) race on it. Each call clears the
-// counters it needs before its kernel runs.
+// status word before its kernels run.
 #include <mutex>
 
 #include "awq_internal.cuh"
@@ -75,10 +76,9 @@ extern "C" awq_status awq_w4a16_gemv_no_alloc(const void* x, const void* qweight
   if (scratch_for_current_device(&scratch) != cudaSuccess) return AWQ_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const GemvPlan p = plan_gemv(M, K, N, d.sm_count);
-  // The status word and the split-K counters must start at zero; the partial
-  // sums are always written before they are read.
-  const size_t zero_bytes = kWsHeaderBytes + round_up((size_t)p.ctas_n * 4, 256);
-  if (cudaMemsetAsync(scratch, 0, zero_bytes, s) != cudaSuccess) return AWQ_ERR_CUDA;
+  // The status word must start at zero; the partial sums are always written
+  // before they are read.
+  if (cudaMemsetAsync(scratch, 0, p.zero_bytes, s) != cudaSuccess) return AWQ_ERR_CUDA;
   cudaError_t e = launch_gemv(static_cast<const __half*>(x), static_cast<const uint32_t*>(qweight),
                               static_cast<const __half*>(scales), static_cast<const uint8_t*>(zeros),
                               static_cast<__half*>(y), M, K, N, scratch, p, s);

@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(512) pack_kernel(const __half* __restrict__ w,
   }
   const uint32_t word = part | __shfl_xor_sync(0xffffffffu, part, 1);
   if ((lane & 1) == 0) {
-    qweight[((nb * KB + kb) * kRowsPerBlock + r) * kWordsPerRow + (lane >> 1)] = word;
+    qweight[(block_index(nb, kb, KB, N / kRowsPerBlock) * kRowsPerBlock + r) * kWordsPerRow + (lane >> 1)] = word;
   }
   if (lane == 0) {
     scales[(int64_t)kb * N + n] = s16;
@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
   const int r = t / kWordsPerRow, wi = t % kWordsPerRow;
   const int64_t KB = K / kKPerBlock;
   const int64_t n = nb * kRowsPerBlock + r;
-  const uint32_t word = qweight[(nb * KB + kb) * kWordsPerBlock + t];
+  const uint32_t word = qweight[block_index(nb, kb, KB, N / kRowsPerBlock) * kWordsPerBlock + t];
   const float s = __half2float(scales[(int64_t)kb * N + n]);
   const int z = (zeros[(int64_t)kb * (N / 2) + (n >> 1)] >> (4 * (n & 1))) & 0xF;
   __align__(16) __half out[8];
