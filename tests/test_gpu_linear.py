@@ -154,6 +154,27 @@ def test_decode_full_size(wl, layer, M):
     check_close(y[:, rows], y_ref, b, f"{wl}/{layer} M={M}")
 
 
+# Shapes whose streamed GEMV unit spans several k-blocks: 4 k-blocks with
+# K/128 = 122 (the last unit of each group has 2) and a last group of 3 row
+# blocks; K/128 = 149 with 4 k-blocks (M <= 3; the last unit has 1) and with
+# 2 k-blocks (M = 8 and 16, where bigger units leave too few ring stages);
+# 4 k-blocks with only 6 k-blocks per group. The checked rows include every
+# row of the first two and the last two groups, where CTA ranges split groups.
+UNIT_CASES = [(15616, 5168, 1), (15616, 5168, 24), (19072, 2048, 1), (19072, 2048, 3), (19072, 2048, 8),
+              (19072, 2048, 16), (768, 75776, 1)]
+
+
+@pytest.mark.parametrize("K,N,M", UNIT_CASES)
+def test_gemv_multi_kblock_units(K, N, M):
+    W, dev, hp = _packed(N, K, f"unit{K}x{N}")
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"unit{K}x{N}/x{M}"), M, K, 1.0)
+    y = _run(awq.awq_w4a16_gemv, x, dev, N)
+    rows = set(sample_rows(N, 64, seed=M).tolist()) | set(range(min(256, N))) | set(range(max(0, N - 256), N))
+    rows = np.array(sorted(rows), dtype=np.int64)
+    y_ref, b = oracle_rows(x, *hp, N, K, rows)
+    check_close(y[:, rows], y_ref, b, f"unit K={K} N={N} M={M}")
+
+
 PREFILL_CASES = [(l.name, M) for l in awq_synth.WORKLOADS["prefill"].layers for M in (512, 2048, 8192)]
 
 

@@ -59,6 +59,9 @@ const DeviceInfo& device_info();   // current device
 // GEMV launch plan (shared by awq_workspace_bytes and the launcher).
 struct GemvPlan {
   int nt;               // token tiles of 8 (1, 2 or 4)
+  int ku;               // k-blocks per streamed unit (1, 2 or 4)
+  int stages;           // depth of the shared-memory ring
+  size_t smem_bytes;    // dynamic shared memory per CTA
   int ctas;             // persistent CTAs (up to two per SM)
   int groups;           // groups of 8 row blocks
   bool has_split;       // some group is split between CTAs (the fixup kernel runs)

@@ -4,34 +4,36 @@
 // (or a few) per step through 4-bit-weight linear layers, so each layer is a
 // GEMV whose cost is streaming its packed weights from HBM once.
 //
-// Work split ("stream-K" over units). A unit is one k-block (128 input
-// channels, one quantization group) of one group of 8 row blocks (128 output
-// channels): R <= 8 KiB of codes that the packed layout stores contiguously,
-// plus their 16R scales and 8R zero bytes. Units are numbered group-major,
-// k-block-minor, i.e. in memory order, and every CTA (two per SM, one for
-// M > 16) streams an equal contiguous range of them, so the load is balanced
-// to one unit.
+// Work split ("stream-K" over units). A unit is KU consecutive k-blocks (128
+// input channels each, one quantization group) of one group of 8 row blocks
+// (128 output channels): up to KU x 8 KiB of codes that the packed layout
+// stores contiguously, plus their scales and zeros (one 256-byte and one
+// 64-byte row slice per k-block). The last unit of a group is shorter when KU
+// does not divide K/128. Units are numbered group-major, i.e. in memory order,
+// and every CTA (two per SM, one for M > 16) streams an equal contiguous
+// range of them, so the load is balanced to one unit. KU (1, 2 or 4) is
+// chosen per layer: bigger units spend less of the producer's issue time on
+// the small per-unit copies, smaller units balance small layers better.
 //
 // Inside a CTA:
-//   warp 0 (producer) keeps an 8-deep shared-memory ring full: per unit one
+//   warp 0 (producer) keeps a ring of shared-memory stages full: per unit one
 //     1-D bulk copy of the codes, cp.async copies of the scales and zeros,
-//     and one 256-byte bulk copy per token of x[m][128 kb .. 128 kb + 127];
-//     completion is tracked by the stage's mbarrier (transaction bytes plus
-//     the cp.async arrivals). The codes of the first eight units are requested
-//     before the kernel waits for the previous grid in the stream
-//     (programmatic dependent launch): they do not depend on it; x does.
+//     and one bulk copy per token of x[m][128 kb0 .. 128 (kb0 + KU)); the
+//     stage's mbarrier tracks completion (transaction bytes plus the cp.async
+//     arrivals). The ring depth follows from the shared memory left for the
+//     stage size. The codes of the first stages are requested before the
+//     kernel waits for the previous grid in the stream (programmatic
+//     dependent launch): they do not depend on it; x does.
 //   warps 1-8 (consumers): warp w owns row block w of every unit, so it
 //     accumulates its 16 output channels over the whole k-range in registers
-//     with no cross-warp reduction. Per unit a lane reads two 16-byte words of
-//     codes (rows g and g+8, k = 32t .. 32t+31), turns them into exact fp16
-//     (q - z) with one lop3 per pair plus hsub2 / hfma2 (the exponent trick:
-//     (word & 0x000F000F) | 0x64006400 is half2(1024 + q_a, 1024 + q_b)), and
-//     feeds mma.sync m16n8k16 (A = 16 rows x 16 k from registers, B = 16 k x 8
-//     tokens from shared memory). The MMA sums over k, so any permutation of k
-//     applied to A and B alike is allowed: a lane pairs the k it loaded
-//     (32t + 8j + 0..3 for MMA 2j, + 4..7 for MMA 2j+1) with the fragment
-//     slots it owns. The fp32 result of a unit is sum_k x (q - z) over one
+//     with no cross-warp reduction. Per k-block a lane reads two 16-byte words
+//     of codes (rows g and g+8, k = 32t .. 32t+31) and feeds mma.sync
+//     m16n8k16 (A = 16 rows x 16 k from registers, B = 16 k x 8 tokens from
+//     shared memory). The MMA sums over k, so any permutation of k applied to
+//     A and B alike is allowed: a lane pairs the k it loaded with the fragment
+//     slots it owns. The fp32 result of a k-block is sum_k x (q - z) over one
 //     group; y += s * that, in fp32, so no weight is rounded.
+//   warp 9 (M <= 8 only): per-k-block sums of x, see block_mma_lohi.
 //
 // Output. A warp that saw all k-blocks of its row block writes fp16 y. A row
 // block split between CTAs (only the first and the last group of a CTA's
@@ -39,6 +41,8 @@
 // plain stores, so streaming never waits on another CTA; a small fixup
 // kernel launched right behind the GEMV (programmatic dependent launch) adds
 // the slots in CTA order (deterministic) and writes y.
+#include <type_traits>
+
 #include "awq_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -46,26 +50,31 @@ namespace awq {
 namespace {
 
 constexpr int kConsumers = kGroupBlocks;  // one consumer warp per row block of a unit
-constexpr int kWarpXsum = 1 + kConsumers;  // per-unit sums of x (M <= 8)
+constexpr int kWarpXsum = 1 + kConsumers;  // per-k-block sums of x (M <= 8)
 constexpr int kThreads = (2 + kConsumers) * 32;
-constexpr int kStages = 8;
-constexpr int kUnitQBytes = kGroupBlocks * 1024;
-constexpr int kUnitScaleBytes = kGroupBlocks * kRowsPerBlock * 2;  // 256
-constexpr int kUnitZeroBytes = kGroupBlocks * kRowsPerBlock / 2;   // 64
-constexpr int kXRowBytes = kKPerBlock * 2;                          // 256
+constexpr int kMaxStages = 16;
+constexpr int kKbQBytes = kGroupBlocks * 1024;                    // codes of one k-block of a group
+constexpr int kKbScaleBytes = kGroupBlocks * kRowsPerBlock * 2;   // 256
+constexpr int kKbZeroBytes = kGroupBlocks * kRowsPerBlock / 2;    // 64
+constexpr int kKbXsBytes = 8 * 2 * 4;                             // 8 tokens x (C, X) fp32
+constexpr int kXRowBytes = kKPerBlock * 2;                        // 256 bytes of x per token and k-block
+// Shared memory one CTA may use (two CTAs per SM share 228 KiB, minus the
+// 1 KiB per CTA the hardware reserves).
+constexpr int kSmemPerCta2 = 112 * 1024;
+constexpr int kSmemPerCta1 = 226 * 1024;
 
-template <int NT>
-struct Layout {
-  static constexpr int kQOff = 0;
-  static constexpr int kSOff = kQOff + kUnitQBytes;
-  static constexpr int kZOff = kSOff + kUnitScaleBytes;
-  static constexpr int kXSOff = kZOff + kUnitZeroBytes;  // per token: C = 1024 X_lo + 64 X_hi, X = X_lo + X_hi
-  static constexpr int kXOff = kXSOff + 8 * 2 * 4;
-  static constexpr int kStageBytes = kXOff + 8 * NT * kXRowBytes;
-  static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kMiscOff = kBarOff + 3 * kStages * 8;  // full, empty, x_landed
-  static constexpr int kBytes = kMiscOff + 16;
-  static_assert(kStageBytes % 16 == 0, "stages must stay 16-byte aligned");
+// Byte offsets inside one ring stage for a unit of up to KU k-blocks and M
+// tokens (the same numbers on the host and in every thread).
+struct Stage {
+  int q, s, z, xs, x, bytes;
+  __host__ __device__ Stage(int KU, int M) {
+    q = 0;
+    s = q + KU * kKbQBytes;
+    z = s + KU * kKbScaleBytes;
+    xs = z + KU * kKbZeroBytes;
+    x = xs + KU * kKbXsBytes;
+    bytes = x + M * KU * kXRowBytes;  // every term is a multiple of 16
+  }
 };
 
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
@@ -76,6 +85,7 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
+// d += A B (m16n8k16, fp16 inputs, fp32 accumulate).
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -84,17 +94,26 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// d = A B (the accumulator input is zero; no separate clearing of d).
+__device__ __forceinline__ void mma_16816_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
 
-// Independent accumulator chains per token tile: the 8 MMAs of a unit are
-// spread over kChains accumulators so that consecutive MMAs do not wait on
+// Independent accumulator chains per token tile: the 8 MMAs of a k-block are
+// spread over Chains accumulators so that consecutive MMAs do not wait on
 // each other's results.
 template <int NT>
 struct Chains {
   static constexpr int value = NT == 1 ? 4 : 2;
 };
 
-// acc[c][nt] += (q - z) * x over one unit's 128 k (split over the chains c),
-// rows g and g+8.
+// acc[c][nt] = (q - z) * x over one k-block (split over the chains c), rows g
+// and g+8 (M > 8).
 template <int NT>
 __device__ __forceinline__ void block_mma(float (&acc)[Chains<NT>::value][NT][4], const uint4& wa4, const uint4& wb4,
                                           uint32_t za, uint32_t zb, const uint4 (&xf)[NT][4]) {
@@ -118,11 +137,15 @@ __device__ __forceinline__ void block_mma(float (&acc)[Chains<NT>::value][NT][4]
       const uint32_t a1 = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(b, kMaskLo, kMagic)), zlo_b));
       const uint32_t a2 = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(a, kMaskHi, kMagic)), sixteenth, zhi_a));
       const uint32_t a3 = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(b, kMaskHi, kMagic)), sixteenth, zhi_b));
+      const int idx = 2 * j + half;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const uint32_t b0 = half ? xf[nt][j].z : xf[nt][j].x;
         const uint32_t b1 = half ? xf[nt][j].w : xf[nt][j].y;
-        mma_16816(acc[(2 * j + half) % C][nt], a0, a1, a2, a3, b0, b1);
+        if (idx < C)
+          mma_16816_first(acc[idx][nt], a0, a1, a2, a3, b0, b1);
+        else
+          mma_16816(acc[idx % C][nt], a0, a1, a2, a3, b0, b1);
       }
       a >>= 8;
       b >>= 8;
@@ -134,15 +157,15 @@ __device__ __forceinline__ void block_mma(float (&acc)[Chains<NT>::value][NT][4]
 // subnormal inputs: the 15 value bits shifted into place read as fp32 are the
 // value times 2^-112.
 __device__ __forceinline__ float pos_half_bits_to_float(uint32_t h) {
-  return __uint_as_float((h & 0x7FFFu) << 13) * 5.192296858534828e+33f;  // 2^112
+  return __uint_as_float(h << 13) * 5.192296858534828e+33f;  // 2^112; the sign bit of h is 0
 }
 
 // M <= 8 (one token tile): the codes go into the MMA unchanged, as the fp16
 // values 1024 + q (pairs taken with the 0x000F000F mask, "lo" k) and
 // 1024 + 16 q (0x00F000F0 mask, "hi" k), in separate MMAs so that the two
-// offsets can be removed afterwards with per-unit sums of x:
+// offsets can be removed afterwards with per-k-block sums of x:
 //   sum_k x (q - z) = acc_lo + acc_hi / 16 - (1024 X_lo + 64 X_hi) - z (X_lo + X_hi)
-// with X_lo, X_hi the sums of x over the lo and hi k of the unit. This needs
+// with X_lo, X_hi the sums of x over the lo and hi k of the k-block. This needs
 // 5 integer ops per 8 weights and no fp16 arithmetic. acc[0..1] are lo chains,
 // acc[2..3] hi chains.
 __device__ __forceinline__ void block_mma_lohi(float (&acc)[4][4], const uint4& wa4, const uint4& wb4,
@@ -154,45 +177,60 @@ __device__ __forceinline__ void block_mma_lohi(float (&acc)[4][4], const uint4& 
   for (int j = 0; j < 4; ++j) {
     const uint32_t a = wa[j], b = wb[j], a8 = wa[j] >> 8, b8 = wb[j] >> 8;
     // slots (2t, 2t+1) <- k = 8j + 0, 1 (lo) / 2, 3 (hi); slots (2t+8, 2t+9) <- 4, 5 / 6, 7
-    mma_16816(acc[j & 1], lop3_and_or(a, kMaskLo, kMagic), lop3_and_or(b, kMaskLo, kMagic),
-              lop3_and_or(a8, kMaskLo, kMagic), lop3_and_or(b8, kMaskLo, kMagic), xf[j].x, xf[j].z);
-    mma_16816(acc[2 + (j & 1)], lop3_and_or(a, kMaskHi, kMagic), lop3_and_or(b, kMaskHi, kMagic),
-              lop3_and_or(a8, kMaskHi, kMagic), lop3_and_or(b8, kMaskHi, kMagic), xf[j].y, xf[j].w);
+    const uint32_t l0 = lop3_and_or(a, kMaskLo, kMagic), l1 = lop3_and_or(b, kMaskLo, kMagic);
+    const uint32_t l2 = lop3_and_or(a8, kMaskLo, kMagic), l3 = lop3_and_or(b8, kMaskLo, kMagic);
+    const uint32_t h0 = lop3_and_or(a, kMaskHi, kMagic), h1 = lop3_and_or(b, kMaskHi, kMagic);
+    const uint32_t h2 = lop3_and_or(a8, kMaskHi, kMagic), h3 = lop3_and_or(b8, kMaskHi, kMagic);
+    if (j < 2) {
+      mma_16816_first(acc[j], l0, l1, l2, l3, xf[j].x, xf[j].z);
+      mma_16816_first(acc[2 + j], h0, h1, h2, h3, xf[j].y, xf[j].w);
+    } else {
+      mma_16816(acc[j & 1], l0, l1, l2, l3, xf[j].x, xf[j].z);
+      mma_16816(acc[2 + (j & 1)], h0, h1, h2, h3, xf[j].y, xf[j].w);
+    }
   }
 }
 
+// Unit numbering: UPG = ceil(KB / KU) units per group; unit u is group
+// u / UPG, k-blocks KU (u % UPG) .. min(KB, KU (u % UPG + 1)) - 1. CTA c of P
+// streams units [c U / P, (c + 1) U / P).
 struct Range {
-  int64_t KB, NB, U, P;
-  __device__ __forceinline__ int64_t first_unit(int64_t c) const { return c * U / P; }
-  __device__ __forceinline__ int64_t cta_of(int64_t u) const { return ((u + 1) * P - 1) / U; }
+  int64_t KB, NB, UPG, U, P;
+  __host__ __device__ Range(int64_t K, int64_t N, int KU, int64_t P_) {
+    KB = K / kKPerBlock;
+    NB = N / kRowsPerBlock;
+    UPG = (KB + KU - 1) / KU;
+    U = (NB + kGroupBlocks - 1) / kGroupBlocks * UPG;
+    P = P_;
+  }
+  __host__ __device__ __forceinline__ int64_t first_unit(int64_t c) const { return c * U / P; }
+  __host__ __device__ __forceinline__ int64_t cta_of(int64_t u) const { return ((u + 1) * P - 1) / U; }
 };
 
-template <int NT>
+// kM1: M == 1 (NT == 1), where only the epilogue slots of token 0 are computed.
+template <int NT, int KU, bool kM1>
 __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
     gemv_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight, const __half* __restrict__ scales,
-                const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M, int K, int N,
+                const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M, int K, int N, int NS,
                 float* __restrict__ partial, uint32_t* status) {
-  using L = Layout<NT>;
   extern __shared__ __align__(16) uint8_t smem[];
-  const uint32_t sbase = ptx::smem_u32(smem);
-  auto full = [&](int s) -> uint32_t { return sbase + L::kBarOff + 8 * s; };
-  auto empty = [&](int s) -> uint32_t { return sbase + L::kBarOff + 8 * (kStages + s); };
-  auto xland = [&](int s) -> uint32_t { return sbase + L::kBarOff + 8 * (2 * kStages + s); };
   constexpr bool kLoHi = NT == 1;
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff);
+  const Stage L(KU, M);
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const uint32_t bar0 = sbase + NS * L.bytes;
+  auto full = [&](int s) -> uint32_t { return bar0 + 8 * s; };
+  auto empty = [&](int s) -> uint32_t { return bar0 + 8 * (kMaxStages + s); };
+  auto xland = [&](int s) -> uint32_t { return bar0 + 8 * (2 * kMaxStages + s); };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + NS * L.bytes + 3 * kMaxStages * 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  Range rg;
-  rg.KB = K / kKPerBlock;
-  rg.NB = N / kRowsPerBlock;
-  rg.U = (rg.NB + kGroupBlocks - 1) / kGroupBlocks * rg.KB;
-  rg.P = gridDim.x;
+  const Range rg(K, N, KU, gridDim.x);
   const int64_t c = blockIdx.x;
   const int64_t u0 = rg.first_unit(c), u1 = rg.first_unit(c + 1);
   const int n_units = (int)(u1 - u0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       // 32 cp.async arrivals + 1 arrival carrying the byte count (+ 1 from the x-sum warp)
       ptx::mbar_init(full(s), kLoHi ? 34 : 33);
       ptx::mbar_init(empty(s), kConsumers);
@@ -207,91 +245,117 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
     // Two cursors walk the CTA's units in order: one for the codes (group,
-    // k-block), one for the activations (k-block only).
-    int64_t cgi = u0 / rg.KB, ckb = u0 % rg.KB, xkb = u0 % rg.KB;
-    auto issue_codes = [&](int i) {  // codes, scales, zeros of unit u0 + i; arms the stage
-      const int s = i % kStages;
+    // unit within the group), one for the activations (unit within the group).
+    int64_t cgi = u0 / rg.UPG;
+    int cj = (int)(u0 % rg.UPG), xj = cj;
+    auto issue_codes = [&](int s) {  // codes, scales, zeros of the next unit into stage s; arms it
       const int R = (int)group_rows(cgi, rg.NB);
-      const uint32_t st = sbase + s * L::kStageBytes;
-      if (lane == 0) ptx::mbar_arrive_expect_tx(full(s), (uint32_t)(R * 1024 + (kLoHi ? 0 : M * kXRowBytes)));
+      const int64_t kb0 = (int64_t)cj * KU;
+      const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
+      const uint32_t st = sbase + s * L.bytes;
+      if (lane == 0)
+        ptx::mbar_arrive_expect_tx(full(s), (uint32_t)(ku * R * 1024 + (kLoHi ? 0 : M * ku * kXRowBytes)));
       __syncwarp();
       if (lane == 0)
-        ptx::bulk_g2s(st + L::kQOff, qweight + unit_first_block(cgi, ckb, rg.KB, rg.NB) * kWordsPerBlock,
-                      (uint32_t)(R * 1024), full(s));
-      if (lane < 2 * R)
-        ptx::cp_async_16(st + L::kSOff + 16 * lane, scales + ckb * N + kGroupBlocks * kRowsPerBlock * cgi + 8 * lane);
-      else if (lane >= 16 && lane < 16 + R)
-        ptx::cp_async_8(st + L::kZOff + 8 * (lane - 16), zeros + ckb * (N / 2) + 64 * cgi + 8 * (lane - 16));
+        ptx::bulk_g2s(st + L.q, qweight + unit_first_block(cgi, kb0, rg.KB, rg.NB) * kWordsPerBlock,
+                      (uint32_t)(ku * R * 1024), full(s));
+      const __half* srow = scales + kb0 * N + kGroupBlocks * kRowsPerBlock * cgi;
+      for (int p = lane; p < ku * 16; p += 32) {  // ku rows of 32 R bytes
+        const int j = p >> 4, l = p & 15;
+        if (l < 2 * R) ptx::cp_async_16(st + L.s + j * kKbScaleBytes + 16 * l, srow + (int64_t)j * N + 8 * l);
+      }
+      const uint8_t* zrow = zeros + kb0 * (N / 2) + 64 * cgi;
+      for (int p = lane; p < ku * 8; p += 32) {  // ku rows of 8 R bytes
+        const int j = p >> 3, l = p & 7;
+        if (l < R) ptx::cp_async_8(st + L.z + j * kKbZeroBytes + 8 * l, zrow + (int64_t)j * (N / 2) + 8 * l);
+      }
       ptx::cp_async_arrive_noinc(full(s));
-      if (++ckb == rg.KB) {
-        ckb = 0;
+      if (++cj == rg.UPG) {
+        cj = 0;
         ++cgi;
       }
     };
-    auto issue_x = [&](int i) {  // activations of unit u0 + i
-      const int s = i % kStages;
+    auto issue_x = [&](int s) {  // activations of the next unit into stage s
+      const int64_t kb0 = (int64_t)xj * KU;
+      const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
       // with the lo/hi split x lands on its own barrier: the x-sum warp reads it first
       const uint32_t xb = kLoHi ? xland(s) : full(s);
       if (kLoHi) {
-        if (lane == 0) ptx::mbar_arrive_expect_tx(xb, (uint32_t)(M * kXRowBytes));
+        if (lane == 0) ptx::mbar_arrive_expect_tx(xb, (uint32_t)(M * ku * kXRowBytes));
         __syncwarp();
       }
       if (lane < M)
-        ptx::bulk_g2s(sbase + s * L::kStageBytes + L::kXOff + kXRowBytes * lane,
-                      x + (int64_t)lane * K + xkb * kKPerBlock, kXRowBytes, xb);
-      if (++xkb == rg.KB) xkb = 0;
+        ptx::bulk_g2s(sbase + s * L.bytes + L.x + KU * kXRowBytes * lane, x + (int64_t)lane * K + kb0 * kKPerBlock,
+                      (uint32_t)(ku * kXRowBytes), xb);
+      if (++xj == rg.UPG) xj = 0;
     };
-    const int pro = n_units < kStages ? n_units : kStages;
+    const int pro = n_units < NS ? n_units : NS;
     for (int i = 0; i < pro; ++i) issue_codes(i);  // independent of the previous grid
     ptx::griddep_wait();
     for (int i = 0; i < pro; ++i) issue_x(i);
-    int i = pro;
+    // unit i goes to stage s = i % NS as its use ph = (i / NS) & 1 and waits
+    // for the consumers' release of the stage's previous use (parity ph ^ 1)
+    int i = pro, s = pro % NS, ph = pro / NS;
     for (; i < n_units; ++i) {
-      const int s = i % kStages;
       bool ok = true;
-      if (lane == 0) ok = ptx::wait_bar(empty(s), ((i / kStages) & 1) ^ 1, abort_flag, status);
+      if (lane == 0) ok = ptx::wait_bar(empty(s), ph ^ 1, abort_flag, status);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      issue_codes(i);
-      issue_x(i);
+      issue_codes(s);
+      issue_x(s);
+      if (++s == NS) {
+        s = 0;
+        ph ^= 1;
+      }
     }
     if (i < n_units && lane == 0)  // aborting: let the copies already issued land
-      for (int j = (i > kStages ? i - kStages : 0); j < i; ++j) ptx::drain_bar(full(j % kStages), (j / kStages) & 1);
+      for (int j = (i > NS ? i - NS : 0); j < i; ++j) ptx::drain_bar(full(j % NS), (j / NS) & 1);
     __syncwarp();
     return;
   }
 
   if (warp == kWarpXsum) {
     // ------------------------------ x sums (M <= 8) ------------------------------
-    // Lane (m, t4) = (lane / 4, lane % 4) adds token m's x over k = 32 t4 .. 32 t4 + 31
-    // into lo (k % 8 in {0, 1, 4, 5}) and hi (k % 8 in {2, 3, 6, 7}) fp32 sums.
+    // Per k-block j of the unit, lane (m, t4) = (lane / 4, lane % 4) adds token
+    // m's x over k = 32 t4 .. 32 t4 + 31 into lo (k % 8 in {0, 1, 4, 5}) and hi
+    // (k % 8 in {2, 3, 6, 7}) fp32 sums.
     if (kLoHi) {
       const int m = lane >> 2, t4 = lane & 3;
+      int jj = (int)(u0 % rg.UPG), s = 0, ph = 0;
       for (int i = 0; i < n_units; ++i) {
-        const int s = i % kStages;
-        if (!ptx::wait_bar(xland(s), (i / kStages) & 1, abort_flag, status)) break;
-        const uint8_t* st = smem + s * L::kStageBytes;
-        float lo = 0.f, hi = 0.f;
-        if (m < M) {
+        if (!ptx::wait_bar(xland(s), ph, abort_flag, status)) break;
+        const int64_t kb0 = (int64_t)jj * KU;
+        const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
+        const uint8_t* st = smem + s * L.bytes;
+        for (int j = 0; j < ku; ++j) {
+          float lo = 0.f, hi = 0.f;
+          if (m < M) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(st + L::kXOff + m * kXRowBytes + 64 * t4 + 16 * j);
-            const float2 p0 = __half22float2(u32_as_h2(v.x)), p1 = __half22float2(u32_as_h2(v.y));
-            const float2 p2 = __half22float2(u32_as_h2(v.z)), p3 = __half22float2(u32_as_h2(v.w));
-            lo += (p0.x + p0.y) + (p2.x + p2.y);
-            hi += (p1.x + p1.y) + (p3.x + p3.y);
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v = *reinterpret_cast<const uint4*>(st + L.x + m * KU * kXRowBytes + j * kXRowBytes +
+                                                              64 * t4 + 16 * q);
+              const float2 p0 = __half22float2(u32_as_h2(v.x)), p1 = __half22float2(u32_as_h2(v.y));
+              const float2 p2 = __half22float2(u32_as_h2(v.z)), p3 = __half22float2(u32_as_h2(v.w));
+              lo += (p0.x + p0.y) + (p2.x + p2.y);
+              hi += (p1.x + p1.y) + (p3.x + p3.y);
+            }
           }
-        }
-        lo += __shfl_xor_sync(0xffffffffu, lo, 1);
-        hi += __shfl_xor_sync(0xffffffffu, hi, 1);
-        lo += __shfl_xor_sync(0xffffffffu, lo, 2);
-        hi += __shfl_xor_sync(0xffffffffu, hi, 2);
-        if (t4 == 0 && m < M) {
-          float* xs = reinterpret_cast<float*>(smem + s * L::kStageBytes + L::kXSOff);
-          xs[2 * m] = 1024.f * lo + 64.f * hi;
-          xs[2 * m + 1] = lo + hi;
+          lo += __shfl_xor_sync(0xffffffffu, lo, 1);
+          hi += __shfl_xor_sync(0xffffffffu, hi, 1);
+          lo += __shfl_xor_sync(0xffffffffu, lo, 2);
+          hi += __shfl_xor_sync(0xffffffffu, hi, 2);
+          if (t4 == 0 && m < M) {
+            float* xs = reinterpret_cast<float*>(smem + s * L.bytes + L.xs + j * kKbXsBytes);
+            xs[2 * m] = 1024.f * lo + 64.f * hi;
+            xs[2 * m + 1] = lo + hi;
+          }
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(full(s));
+        if (++jj == rg.UPG) jj = 0;
+        if (++s == NS) {
+          s = 0;
+          ph ^= 1;
+        }
       }
     }
     return;
@@ -304,9 +368,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
   int64_t cur_gi = -1;
 
   // ---- output of one row block ----
-  auto covered = [&](int64_t g_) { return u0 <= g_ * rg.KB && (g_ + 1) * rg.KB <= u1; };
+  auto covered = [&](int64_t g_) { return u0 <= g_ * rg.UPG && (g_ + 1) * rg.UPG <= u1; };
   auto write_y = [&](int64_t g_, const float (&v)[NT][4]) {
-    if (cw >= group_rows(g_, rg.NB)) return;
     const int64_t ra = (g_ * kGroupBlocks + cw) * kRowsPerBlock + g;  // rows ra (c = 0, 1), ra + 8 (c = 2, 3)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -318,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
   };
   // Partial slot of CTA `cta` for group g_: [cta][first/last group of cta][row block][16 rows][M].
   auto slot = [&](int64_t cta, int64_t g_) -> float* {
-    const int which = (g_ == rg.first_unit(cta) / rg.KB) ? 0 : 1;
+    const int which = (g_ == rg.first_unit(cta) / rg.UPG) ? 0 : 1;
     return partial + ((cta * 2 + which) * kGroupBlocks + cw) * kRowsPerBlock * M;
   };
   auto store_partial = [&](int64_t g_, const float (&v)[NT][4]) {
@@ -341,12 +404,87 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       store_partial(g_, v);
   };
 
+  // ---- one k-block (index j of the unit in stage st) of this warp's row block ----
+  // kb_issue loads the k-block, issues its MMAs into `acc` and keeps in `ks`
+  // what the epilogue needs besides the MMA results; kb_finish adds the
+  // k-block to yacc. (Finishing a k-block only after the next one's MMAs were
+  // issued measured no faster on B200.)
+  constexpr int kC = Chains<NT>::value;
+  using Acc = std::conditional_t<kLoHi, float[4][4], float[kC][NT][4]>;
+  struct KState {
+    float s[2];     // scales of rows g, g + 8
+    float corr[4];  // lo/hi path: s (C + z X) of slot cc (rows g / g+8, tokens 2t / 2t+1)
+  };
+  auto kb_issue = [&](const uint8_t* st, int j, int R, Acc& acc, KState& ks) {
+    const uint8_t* blk = st + L.q + (j * R + cw) * 1024;
+    const uint4 wa = *reinterpret_cast<const uint4*>(blk + g * 64 + 16 * t);
+    const uint4 wb = *reinterpret_cast<const uint4*>(blk + (g + 8) * 64 + 16 * t);
+    const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + L.s + j * kKbScaleBytes) + cw * kRowsPerBlock;
+    ks.s[0] = pos_half_bits_to_float(sc[g]);
+    ks.s[1] = pos_half_bits_to_float(sc[g + 8]);
+    const uint8_t* zr = st + L.z + j * kKbZeroBytes + cw * (kRowsPerBlock / 2);
+    const uint32_t za = (zr[g >> 1] >> (4 * (g & 1))) & 0xF;
+    const uint32_t zb = (zr[(g + 8) >> 1] >> (4 * (g & 1))) & 0xF;
+    uint4 xf[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int m = 8 * nt + g;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        xf[nt][q] = m < M ? *reinterpret_cast<const uint4*>(st + L.x + (m * KU + j) * kXRowBytes + 64 * t + 16 * q)
+                          : make_uint4(0, 0, 0, 0);
+    }
+    if constexpr (kLoHi) {
+      block_mma_lohi(acc, wa, wb, xf[0]);
+      // C and X of tokens 2t and 2t + 1
+      const float4 cx = *reinterpret_cast<const float4*>(st + L.xs + j * kKbXsBytes + 16 * t);
+      const float zf[2] = {__uint_as_float(0x4B000000u | za) - 8388608.f,  // exact (float)z
+                           __uint_as_float(0x4B000000u | zb) - 8388608.f};
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        if (kM1 && (cc & 1)) continue;  // slots of token 1
+        const float Cm = (cc & 1) ? cx.z : cx.x, Xm = (cc & 1) ? cx.w : cx.y;
+        ks.corr[cc] = ks.s[cc >> 1] * fmaf(zf[cc >> 1], Xm, Cm);
+      }
+    } else {
+      block_mma<NT>(acc, wa, wb, za, zb, xf);
+    }
+  };
+  auto kb_finish = [&](const Acc& acc, const KState& ks) {
+    if constexpr (kLoHi) {
+      // y += s (acc_lo + acc_hi / 16) - s (C + z X)
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        if (kM1 && (cc & 1)) continue;
+        const float lo = acc[0][cc] + acc[1][cc], hi = acc[2][cc] + acc[3][cc];
+        yacc[0][cc] = fmaf(ks.s[cc >> 1], fmaf(hi, 0.0625f, lo), yacc[0][cc]) - ks.corr[cc];
+      }
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float v = acc[0][nt][cc];
+#pragma unroll
+          for (int ch = 1; ch < kC; ++ch) v += acc[ch][nt][cc];
+          yacc[nt][cc] = fmaf(ks.s[cc >> 1], v, yacc[nt][cc]);
+        }
+    }
+  };
+
+  auto kblock = [&](const uint8_t* st, int j, int R) {
+    Acc acc;
+    KState ks;
+    kb_issue(st, j, R, acc, ks);
+    kb_finish(acc, ks);
+  };
+
   bool ok = true;
-  int64_t gi = u0 / rg.KB, kb = u0 % rg.KB;  // unit u0 + i is (gi, kb)
-  for (int i = 0; i < n_units; ++i, ++kb) {
-    const int s = i % kStages;
-    if (kb == rg.KB) {
-      kb = 0;
+  int64_t gi = u0 / rg.UPG;
+  int jj = (int)(u0 % rg.UPG), s = 0, ph = 0, R = 0;
+  for (int i = 0; i < n_units; ++i, ++jj) {
+    if (jj == rg.UPG) {
+      jj = 0;
       ++gi;
     }
     if (gi != cur_gi) {
@@ -356,123 +494,77 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) yacc[nt][cc] = 0.f;
       cur_gi = gi;
+      R = (int)group_rows(gi, rg.NB);
     }
-    if (!ptx::wait_bar(full(s), (i / kStages) & 1, abort_flag, status)) {
+    if (!ptx::wait_bar(full(s), ph, abort_flag, status)) {
       ok = false;
       break;
     }
-    if (cw < group_rows(gi, rg.NB)) {
-      const uint8_t* st = smem + s * L::kStageBytes;
-      const uint8_t* blk = st + L::kQOff + cw * 1024;
-      const uint4 wa = *reinterpret_cast<const uint4*>(blk + g * 64 + 16 * t);
-      const uint4 wb = *reinterpret_cast<const uint4*>(blk + (g + 8) * 64 + 16 * t);
-      const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + L::kSOff) + cw * kRowsPerBlock;
-      const float sa = pos_half_bits_to_float(sc[g]), sb = pos_half_bits_to_float(sc[g + 8]);
-      const uint8_t* zr = st + L::kZOff + cw * (kRowsPerBlock / 2);
-      const uint32_t za = (zr[g >> 1] >> (4 * (g & 1))) & 0xF;
-      const uint32_t zb = (zr[(g + 8) >> 1] >> (4 * (g & 1))) & 0xF;
-      uint4 xf[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int m = 8 * nt + g;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          xf[nt][j] = m < M ? *reinterpret_cast<const uint4*>(st + L::kXOff + m * kXRowBytes + 64 * t + 16 * j)
-                            : make_uint4(0, 0, 0, 0);
-      }
-      if constexpr (kLoHi) {
-        float acc[4][4];
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) acc[ch][cc] = 0.f;
-        block_mma_lohi(acc, wa, wb, xf[0]);
-        // C and X of tokens 2t and 2t + 1
-        const float4 cx = *reinterpret_cast<const float4*>(st + L::kXSOff + 16 * t);
-        const float zfa = __uint_as_float(0x4B000000u | za) - 8388608.f;  // exact (float)z
-        const float zfb = __uint_as_float(0x4B000000u | zb) - 8388608.f;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const float lo = acc[0][cc] + acc[1][cc], hi = acc[2][cc] + acc[3][cc];
-          const float Cm = (cc & 1) ? cx.z : cx.x, Xm = (cc & 1) ? cx.w : cx.y;
-          float v = fmaf(hi, 0.0625f, lo) - Cm;
-          v = fmaf(-(cc < 2 ? zfa : zfb), Xm, v);
-          yacc[0][cc] = fmaf(cc < 2 ? sa : sb, v, yacc[0][cc]);
-        }
+    if (cw < R) {
+      const uint8_t* st = smem + s * L.bytes;
+      const int64_t kb0 = (int64_t)jj * KU;
+      const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
+      if (ku == KU) {
+#pragma unroll 2
+        for (int j = 0; j < KU; ++j) kblock(st, j, R);  // no guard: pairs of k-blocks can interleave
       } else {
-        constexpr int C = Chains<NT>::value;
-        float acc[C][NT][4];
-#pragma unroll
-        for (int ch = 0; ch < C; ++ch)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) acc[ch][nt][cc] = 0.f;
-        block_mma<NT>(acc, wa, wb, za, zb, xf);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            float v = acc[0][nt][cc];
-#pragma unroll
-            for (int ch = 1; ch < C; ++ch) v += acc[ch][nt][cc];
-            yacc[nt][cc] += (cc < 2 ? sa : sb) * v;
-          }
+#pragma unroll 1
+        for (int j = 0; j < ku; ++j) kblock(st, j, R);
       }
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(empty(s));
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1;
+    }
   }
   if (ok && cur_gi >= 0) finish_group(cur_gi, yacc);
 }
 
-// Rows split between CTAs: one CTA per group (128 threads, thread = row),
-// launched right after the GEMV in the same stream. It waits for the GEMV's
-// writes (programmatic dependent launch), adds the contributors' partial
-// slots in CTA order and writes fp16 y. Groups that one CTA covered exit.
+// Rows split between CTAs: one CTA per (group, token) (128 threads, thread =
+// row), launched right after the GEMV in the same stream. It waits for the
+// GEMV's writes (programmatic dependent launch), adds the contributors'
+// partial slots in CTA order and writes fp16 y. Groups that one CTA covered
+// exit.
 __global__ void __launch_bounds__(128) gemv_fixup_kernel(const float* __restrict__ partial, __half* __restrict__ y,
-                                                          int M, int K, int N, int P) {
+                                                          int M, int K, int N, int KU, int P) {
   ptx::griddep_launch_dependents();
-  Range rg;
-  rg.KB = K / kKPerBlock;
-  rg.NB = N / kRowsPerBlock;
-  rg.U = (rg.NB + kGroupBlocks - 1) / kGroupBlocks * rg.KB;
-  rg.P = P;
+  const Range rg(K, N, KU, P);
   const int64_t gi = blockIdx.x;
-  const int64_t c_first = rg.cta_of(gi * rg.KB), c_last = rg.cta_of((gi + 1) * rg.KB - 1);
+  const int64_t c_first = rg.cta_of(gi * rg.UPG), c_last = rg.cta_of((gi + 1) * rg.UPG - 1);
   if (c_first == c_last) return;
   const int rb = threadIdx.x >> 4, row = threadIdx.x & 15;
   if (rb >= group_rows(gi, rg.NB)) return;
+  const int m = blockIdx.y;
   ptx::griddep_wait();
-  for (int m = 0; m < M; ++m) {
-    float v = 0.f;
-    for (int64_t q0 = c_first; q0 <= c_last; q0 += 8) {
-      float part[8];
+  float v = 0.f;
+  for (int64_t q0 = c_first; q0 <= c_last; q0 += 8) {
+    float part[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int64_t q = q0 + k;
-        part[k] = 0.f;
-        if (q <= c_last) {
-          const int which = (gi == rg.first_unit(q) / rg.KB) ? 0 : 1;
-          part[k] = __ldcg(partial + (((q * 2 + which) * kGroupBlocks + rb) * kRowsPerBlock + row) * M + m);
-        }
+    for (int k = 0; k < 8; ++k) {
+      const int64_t q = q0 + k;
+      part[k] = 0.f;
+      if (q <= c_last) {
+        const int which = (gi == rg.first_unit(q) / rg.UPG) ? 0 : 1;
+        part[k] = __ldcg(partial + (((q * 2 + which) * kGroupBlocks + rb) * kRowsPerBlock + row) * M + m);
       }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) v += part[k];
     }
-    y[(int64_t)m * N + gi * kGroupBlocks * kRowsPerBlock + threadIdx.x] = __float2half_rn(v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v += part[k];
   }
+  y[(int64_t)m * N + gi * kGroupBlocks * kRowsPerBlock + threadIdx.x] = __float2half_rn(v);
 }
 
-template <int NT>
+template <int NT, int KU, bool kM1>
 cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros, __half* y,
                      int M, int K, int N, void* workspace, const GemvPlan& p, cudaStream_t stream) {
-  using L = Layout<NT>;
   static uint64_t attr_set = 0;  // one bit per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
   if (!(attr_set >> dev & 1)) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, KU, kM1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         NT == 4 ? kSmemPerCta1 : kSmemPerCta2);
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
   }
@@ -482,34 +574,67 @@ cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* sca
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.ctas);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = L::kBytes;
+  cfg.dynamicSmemBytes = p.smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<NT>, x, qweight, scales, zeros, y, M, K, N, partial, status);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<NT, KU, kM1>, x, qweight, scales, zeros, y, M, K, N, p.stages,
+                                     partial, status);
   if (e != cudaSuccess || !p.has_split) return e;
   cudaLaunchConfig_t fcfg = cfg;
-  fcfg.gridDim = dim3((unsigned)p.groups);
+  fcfg.gridDim = dim3((unsigned)p.groups, (unsigned)M);
   fcfg.blockDim = dim3(kGroupBlocks * kRowsPerBlock);
   fcfg.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&fcfg, gemv_fixup_kernel, (const float*)partial, y, M, K, N, p.ctas);
+  return cudaLaunchKernelEx(&fcfg, gemv_fixup_kernel, (const float*)partial, y, M, K, N, p.ku, p.ctas);
+}
+
+template <int NT, bool kM1>
+cudaError_t launch_nt(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
+                      __half* y, int M, int K, int N, void* workspace, const GemvPlan& p, cudaStream_t stream) {
+  switch (p.ku) {
+    case 1: return launch_t<NT, 1, kM1>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    case 2: return launch_t<NT, 2, kM1>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    case 4: return launch_t<NT, 4, kM1>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    default: return cudaErrorInvalidConfiguration;
+  }
 }
 
 }  // namespace
+
+// Unit size: the largest KU in {4, 2, 1} (at most K/128) that leaves room for
+// kMinStages ring stages and still gives every SM a unit. Measured on B200
+// (LLaMA-2-7B and -70B decode layers, M = 1 and 8), bigger units won even
+// where they leave some CTAs idle: one 32 KiB copy per CTA streams faster
+// than four 8 KiB ones.
+constexpr int kMinStages = 3;
 
 GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int sm_count) {
   GemvPlan p{};
   p.nt = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
   const int64_t NB = N / kRowsPerBlock, KB = K / kKPerBlock;
-  const int64_t U = (NB + kGroupBlocks - 1) / kGroupBlocks * KB;
-  const int64_t per_sm = p.nt == 4 ? 1 : 2;  // resident CTAs per SM (shared memory and registers)
-  p.ctas = (int)(U < per_sm * sm_count ? U : per_sm * sm_count);
   p.groups = (int)((NB + kGroupBlocks - 1) / kGroupBlocks);
-  p.has_split = false;  // does some CTA boundary fall inside a group?
-  for (int64_t cc = 1; cc < p.ctas && !p.has_split; ++cc) p.has_split = (cc * U / p.ctas) % KB != 0;
+  const int64_t per_sm = p.nt == 4 ? 1 : 2;  // resident CTAs per SM (shared memory and registers)
+  const int budget = (p.nt == 4 ? kSmemPerCta1 : kSmemPerCta2) - 3 * kMaxStages * 8 - 16;
+  const int64_t Mi = M < 1 ? 1 : M;
+  for (int ku : {4, 2, 1}) {
+    const int64_t U = p.groups * ((KB + ku - 1) / ku);
+    const int stage = Stage(ku, (int)Mi).bytes;
+    int stages = budget / stage;
+    if (stages > kMaxStages) stages = kMaxStages;
+    const bool last = ku == 1;
+    if (!last && (ku > KB || stages < kMinStages || U < sm_count)) continue;
+    p.ku = ku;
+    p.stages = stages;
+    p.smem_bytes = (size_t)stages * stage + 3 * kMaxStages * 8 + 16;
+    p.ctas = (int)(U < per_sm * sm_count ? U : per_sm * sm_count);
+    const Range rg(K, N, ku, p.ctas);
+    p.has_split = false;  // does some CTA boundary fall inside a group?
+    for (int64_t cc = 1; cc < p.ctas && !p.has_split; ++cc) p.has_split = rg.first_unit(cc) % rg.UPG != 0;
+    break;
+  }
   p.partial_off = kWsHeaderBytes;
   p.zero_bytes = kWsHeaderBytes;  // the status word starts at zero
   p.ws_bytes = p.partial_off + (size_t)p.ctas * 2 * kGroupBlocks * kRowsPerBlock * (size_t)M * 4;
@@ -521,9 +646,11 @@ cudaError_t launch_gemv(const __half* x, const uint32_t* qweight, const __half* 
                         cudaStream_t stream) {
   const int m = (int)M, k = (int)K, n = (int)N;
   switch (p.nt) {
-    case 1: return launch_t<1>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
-    case 2: return launch_t<2>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
-    case 4: return launch_t<4>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
+    case 1:
+      return m == 1 ? launch_nt<1, true>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream)
+                    : launch_nt<1, false>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
+    case 2: return launch_nt<2, false>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
+    case 4: return launch_nt<4, false>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
     default: return cudaErrorInvalidConfiguration;
   }
 }
