@@ -28,11 +28,17 @@
  *   - the packed layout (our own; the pages only name a ".pt" checkpoint):
  *       qweight  uint32, 1 KiB blocks of 16 rows x 128 input channels.
  *                Block (nb, kb) holds rows n = 16nb + r (r = 0..15) and
- *                k = 128kb .. 128kb+127; word w of row r holds
- *                k = 128kb + 8w + i, i = 0..7, with the nibble of even i at
- *                bits 4*(i/2) and of odd i at bits 16 + 4*(i/2).  (So
- *                (word >> 4j) & 0x000F000F holds the adjacent pair
- *                k = 8w+2j, 8w+2j+1 as two 16-bit lanes.)
+ *                k = 128kb .. 128kb+127; word w of row r holds the eight
+ *                inputs k = 128kb + k0(w) + i, i = 0..7, with the nibble of
+ *                even i at bits 4*(i/2) and of odd i at bits 16 + 4*(i/2).
+ *                (So (word >> 4j) & 0x000F000F holds the adjacent pair
+ *                k0+2j, k0+2j+1 as two 16-bit lanes.)  For G = 128 (and any
+ *                multiple of 128) k0(w) = 8w. For G = 64 or 32, with
+ *                w = 4t + j (t, j = 0..3) and J = G/32:
+ *                  k0(w) = G*(j / J) + 8*(t*J + j % J),
+ *                so the four words 4t .. 4t+3 that a GPU lane reads at once
+ *                hold inputs of every group of the k-block, and the four
+ *                words with the same j hold whole groups (group j / J).
  *                Blocks are grouped by 8 row blocks (128 rows): group
  *                gi = nb / 8 has R = min(8, N/16 - 8gi) row blocks and is
  *                stored k-block-major, so block (nb, kb) is block number
@@ -173,10 +179,21 @@ int orc_dequant(const uint8_t* q, const uint8_t* z, const uint16_t* s, int64_t N
 /* Bit position of element i (0..7) inside its 32-bit word. */
 static int nibble_shift(int i) { return (i % 2 == 0) ? 4 * (i / 2) : 16 + 4 * (i / 2); }
 
+/* Word (0..15) of its row that holds input k (0..127) of a k-block, the
+ * inverse of k0(w) above; -1 for a group size the layout does not define. */
+static int word_in_row(int k, int G) {
+  if (G % 128 == 0) return k / 8;
+  if (G != 32 && G != 64) return -1;
+  int J = G / 32;
+  int group = k / G, p = (k % G) / 8;  /* 8-input piece p of group `group` */
+  int t = p / J, j = group * J + p % J;
+  return 4 * t + j;
+}
+
 /* Index of the word holding (n, k): block number (group-major, k-block,
  * row block within the group), then row r and word w inside the block. */
-static int64_t word_index(int64_t n, int64_t k, int64_t K, int64_t N) {
-  int64_t nb = n / 16, r = n % 16, kb = k / 128, w = (k % 128) / 8;
+static int64_t word_index(int64_t n, int64_t k, int64_t K, int64_t N, int G) {
+  int64_t nb = n / 16, r = n % 16, kb = k / 128, w = word_in_row((int)(k % 128), G);
   int64_t gi = nb / 8, NB = N / 16;
   int64_t rows_in_group = (NB - 8 * gi < 8) ? NB - 8 * gi : 8;
   int64_t block = 8 * gi * (K / 128) + kb * rows_in_group + nb % 8;
@@ -185,13 +202,13 @@ static int64_t word_index(int64_t n, int64_t k, int64_t K, int64_t N) {
 
 int orc_pack(const uint8_t* q, const uint8_t* z, const uint16_t* s, int64_t N, int64_t K, int G,
              uint32_t* qweight, uint16_t* scales, uint8_t* zeros) {
-  if (bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  if (bad_shape(N, K, G) || word_in_row(0, G) < 0) return ORC_ERR_SHAPE;
   int64_t ng = K / G;
   memset(qweight, 0, sizeof(uint32_t) * (size_t)(N * K / 8));
   memset(zeros, 0, (size_t)(ng * N / 2));
   for (int64_t n = 0; n < N; ++n)
     for (int64_t k = 0; k < K; ++k)
-      qweight[word_index(n, k, K, N)] |= (uint32_t)(q[n * K + k] & 0xF) << nibble_shift((int)(k % 8));
+      qweight[word_index(n, k, K, N, G)] |= (uint32_t)(q[n * K + k] & 0xF) << nibble_shift((int)(k % 8));
   for (int64_t g = 0; g < ng; ++g)
     for (int64_t n = 0; n < N; ++n) {
       scales[g * N + n] = s[n * ng + g];
@@ -202,11 +219,11 @@ int orc_pack(const uint8_t* q, const uint8_t* z, const uint16_t* s, int64_t N, i
 
 int orc_unpack(const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros, int64_t N, int64_t K,
                int G, uint8_t* q, uint8_t* z, uint16_t* s) {
-  if (bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  if (bad_shape(N, K, G) || word_in_row(0, G) < 0) return ORC_ERR_SHAPE;
   int64_t ng = K / G;
   for (int64_t n = 0; n < N; ++n)
     for (int64_t k = 0; k < K; ++k)
-      q[n * K + k] = (uint8_t)((qweight[word_index(n, k, K, N)] >> nibble_shift((int)(k % 8))) & 0xF);
+      q[n * K + k] = (uint8_t)((qweight[word_index(n, k, K, N, G)] >> nibble_shift((int)(k % 8))) & 0xF);
   for (int64_t g = 0; g < ng; ++g)
     for (int64_t n = 0; n < N; ++n) {
       s[n * ng + g] = scales[g * N + n];
@@ -272,7 +289,7 @@ static void packed_row(const uint32_t* qweight, const uint16_t* scales, const ui
                        int64_t K, int G, int64_t n, double* row) {
   for (int64_t k = 0; k < K; ++k) {
     int64_t g = k / G;
-    uint32_t q = (qweight[word_index(n, k, K, N)] >> nibble_shift((int)(k % 8))) & 0xF;
+    uint32_t q = (qweight[word_index(n, k, K, N, G)] >> nibble_shift((int)(k % 8))) & 0xF;
     uint32_t z = (zeros[g * (N / 2) + n / 2] >> (4 * (n % 2))) & 0xF;
     double s = orc_half_to_double(scales[g * N + n]);
     row[k] = orc_half_to_double(orc_double_to_half(((double)q - (double)z) * s));
@@ -284,7 +301,7 @@ static void packed_row(const uint32_t* qweight, const uint16_t* scales, const ui
 int orc_linear_rows(const uint16_t* x, int64_t M, const uint32_t* qweight, const uint16_t* scales,
                     const uint8_t* zeros, int64_t N, int64_t K, int G, int64_t n0, int64_t n1, double* y,
                     double* bound) {
-  if (M < 0 || bad_shape(N, K, G) || n0 < 0 || n1 > N || n0 > n1) return ORC_ERR_SHAPE;
+  if (M < 0 || bad_shape(N, K, G) || word_in_row(0, G) < 0 || n0 < 0 || n1 > N || n0 > n1) return ORC_ERR_SHAPE;
   int64_t W = n1 - n0;
   double* row = (double*)malloc(sizeof(double) * (size_t)K);
   for (int64_t n = n0; n < n1; ++n) {
@@ -313,7 +330,7 @@ int orc_linear(const uint16_t* x, int64_t M, const uint32_t* qweight, const uint
 int orc_linear_entries(const uint16_t* x, int64_t M, const uint32_t* qweight, const uint16_t* scales,
                        const uint8_t* zeros, int64_t N, int64_t K, int G, const int64_t* ms,
                        const int64_t* ns, int64_t count, double* y, double* bound) {
-  if (M < 0 || bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  if (M < 0 || bad_shape(N, K, G) || word_in_row(0, G) < 0) return ORC_ERR_SHAPE;
   double* row = (double*)malloc(sizeof(double) * (size_t)K);
   int64_t cached = -1;
   for (int64_t i = 0; i < count; ++i) {

@@ -60,8 +60,10 @@ def quant_groups(G=128):
 
 
 def packed_words():
-    """-> list of (N, K, n, k, qvalue, word_index, word_value)."""
+    """-> list of (N, K, n, k, qvalue, word_index, word_value, G); G is 128 where
+    the line gives none."""
     out = []
     for t in _lines("packed_words.txt"):
-        out.append(tuple(int(x, 0) for x in t))
+        v = [int(x, 0) for x in t]
+        out.append(tuple(v + [128] * (8 - len(v))))
     return out

@@ -9,6 +9,7 @@ route through the per-group codes.
 from fractions import Fraction
 
 import numpy as np
+import pytest
 
 import awq_synth
 import oracle
@@ -16,7 +17,7 @@ import oracle
 G = 128
 
 
-def _layer(N, K, tag, std=0.02):
+def _layer(N, K, tag, G=G, std=0.02):
     W = awq_synth.matrix_f16(awq_synth.key(0, 98, f"{tag}/W"), N, K, std)
     q, z, s, _ = oracle.quantize(W, G)
     return q, z, s, oracle.dequant(q, z, s, G)
@@ -77,11 +78,12 @@ def test_small_integer_sums_are_exact():
     assert (y == exact).all()
 
 
-def test_factored_route_agrees_exactly_when_w_hat_is_exact():
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_factored_route_agrees_exactly_when_w_hat_is_exact(G):
     # power-of-two scales make every (q - z) s an exact fp16 value, so the two
     # routes differ only by fp64 summation order
     rng = np.random.default_rng(9)
-    N, K, M = 48, 6 * G, 4
+    N, K, M = 48, (6 * G if 6 * G % 128 == 0 else 8 * G), 4
     q = rng.integers(0, 16, (N, K)).astype(np.uint8)
     z = rng.integers(0, 16, (N, K // G)).astype(np.uint8)
     s = np.exp2(rng.integers(-12, -4, (N, K // G))).astype(np.float16)
@@ -106,9 +108,10 @@ def test_factored_route_within_the_rounding_of_w_hat():
     assert np.abs(y - y2).max() > 0          # the rounding of W^ is visible
 
 
-def test_linear_from_packed_buffers_equals_dequant_then_matmul():
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_linear_from_packed_buffers_equals_dequant_then_matmul(G):
     N, K, M = 32, 4 * G, 3
-    q, z, s, wh = _layer(N, K, "lin")
+    q, z, s, wh = _layer(N, K, "lin", G)
     qw, sc, ze = oracle.pack(q, z, s, G)
     x = awq_synth.matrix_f16(awq_synth.key(0, 98, "lin/x"), M, K, 1.0)
     y, b = oracle.matmul(x, wh)

@@ -6,6 +6,7 @@ it. Dequantization is pinned to numpy's own fp16 rounding of the exact
 product (q - z) s.
 """
 import numpy as np
+import pytest
 
 import oracle
 from golden_io import packed_words
@@ -14,12 +15,12 @@ G = 128
 
 
 def test_single_nibbles_land_on_hand_derived_words():
-    for N, K, n, k, qv, widx, wval in packed_words():
+    for N, K, n, k, qv, widx, wval, g in packed_words():
         q = np.zeros((N, K), np.uint8)
         q[n, k] = qv
-        z = np.zeros((N, K // G), np.uint8)
-        s = np.zeros((N, K // G), np.float16)
-        qw, _, _ = oracle.pack(q, z, s, G)
+        z = np.zeros((N, K // g), np.uint8)
+        s = np.zeros((N, K // g), np.float16)
+        qw, _, _ = oracle.pack(q, z, s, g)
         flat = qw.reshape(-1)
         nz = np.flatnonzero(flat)
         assert list(nz) == [widx], (n, k, nz)
@@ -54,7 +55,8 @@ def test_scale_and_zero_layout():
     assert sc.reshape(-1)[21] == np.float16(1.5) and np.count_nonzero(sc) == 1
 
 
-def test_pack_unpack_round_trips():
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_pack_unpack_round_trips(G):
     rng = np.random.default_rng(11)
     for N, K in [(16, 128), (48, 384), (64, 1024)]:
         q = rng.integers(0, 16, (N, K)).astype(np.uint8)
@@ -71,7 +73,29 @@ def test_pack_unpack_round_trips():
         assert (qw2 == qw_r).all() and (ze2 == ze_r).all() and (sc2.view(np.uint16) == sc.view(np.uint16)).all()
 
 
-def test_dequant_is_numpy_rounding_of_the_exact_product():
+@pytest.mark.parametrize("G", [64, 32])
+def test_words_of_one_group_size_hold_whole_groups(G):
+    """G = 64, 32: the four words 4t .. 4t+3 a GPU lane reads hold one 8-input
+    piece of every group of the k-block, and the words with the same j (word
+    index mod 4) hold whole groups, group j / (G / 32); within a word the eight
+    inputs stay consecutive."""
+    N, K = 16, 128
+    J = G // 32
+    q = np.zeros((N, K), np.uint8)
+    q[:, :] = (np.arange(K) // G + 1)[None, :]          # group index + 1
+    qw, _, _ = oracle.pack(q, np.zeros((N, K // G), np.uint8), np.zeros((N, K // G), np.float16), G)
+    words = qw.reshape(-1)[:16]                          # row 0 of the only block
+    for w, word in enumerate(words):
+        nib = [(int(word) >> sh) & 0xF for sh in (0, 16, 4, 20, 8, 24, 12, 28)]  # i = 0..7
+        assert len(set(nib)) == 1 and nib[0] == (w % 4) // J + 1, (w, hex(int(word)))
+    # consecutive inputs: q = k % 8 shows the order inside every word
+    q[:, :] = (np.arange(K) % 8)[None, :]
+    qw, _, _ = oracle.pack(q, np.zeros((N, K // G), np.uint8), np.zeros((N, K // G), np.float16), G)
+    assert (qw.reshape(-1)[:16] == 0x75316420).all()
+
+
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_dequant_is_numpy_rounding_of_the_exact_product(G):
     rng = np.random.default_rng(5)
     N, K = 32, 4 * G
     q = rng.integers(0, 16, (N, K)).astype(np.uint8)

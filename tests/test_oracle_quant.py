@@ -30,7 +30,7 @@ def test_hand_derived_groups():
                 assert wh[r, i] == bits, (c["name"], i, hex(wh[r, i]), hex(bits))
 
 
-def _exact_groups(rng, N, K):
+def _exact_groups(rng, N, K, G=G):
     """W built from random (q, z, s) with s = m * 2^e (m odd <= 127) and every
     group spanning the whole grid (one q = 0 and one q = 15), so that every
     (q - z) * s is an exact fp16 value, hi - lo = 15 s and R / 15 = s exactly."""
@@ -51,9 +51,10 @@ def _exact_groups(rng, N, K):
     return W, q, z, s
 
 
-def test_exactly_representable_weights_have_zero_error():
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_exactly_representable_weights_have_zero_error(G):
     rng = np.random.default_rng(7)
-    W, q0, z0, s0 = _exact_groups(rng, 64, 4 * G)
+    W, q0, z0, s0 = _exact_groups(rng, 64, 4 * G, G)
     q, z, s, _ = oracle.quantize(W, G)
     assert (q == q0).all()
     assert (z == z0).all()
@@ -62,7 +63,7 @@ def test_exactly_representable_weights_have_zero_error():
     assert (wh.view(np.uint16) == W.view(np.uint16)).all()
 
 
-def _random_weights():
+def _random_weights(G=G):
     """Seeded weights with the value mixes the kernels meet: N(0, 0.02),
     outlier channels x20, all-positive and all-negative groups, groups whose
     range is so small that the scale is subnormal, and constant groups."""
@@ -79,17 +80,19 @@ def _random_weights():
     return W.astype(np.float16)
 
 
-def test_codes_and_zero_points_in_range():
-    q, z, s, _ = oracle.quantize(_random_weights(), G)
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_codes_and_zero_points_in_range(G):
+    q, z, s, _ = oracle.quantize(_random_weights(G), G)
     assert q.max() <= 15 and z.max() <= 15
     assert (s.astype(np.float64) > 0).all()
 
 
-def test_every_code_is_a_nearest_grid_point():
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_every_code_is_a_nearest_grid_point(G):
     """Brute force over the 16 codes: (q - z) s is a nearest point of the
     group's grid {(c - z) s : c = 0..15} to v, and exact ties go to even
     q - z (round half to even)."""
-    W = _random_weights()
+    W = _random_weights(G)
     q, z, s, _ = oracle.quantize(W, G)
     N, K = W.shape
     v = W.astype(np.float64)
@@ -106,8 +109,9 @@ def test_every_code_is_a_nearest_grid_point():
     assert (d % 2 == 0).all()
 
 
-def test_scale_is_range_over_15_and_zero_point_centres_the_minimum():
-    W = _random_weights()
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_scale_is_range_over_15_and_zero_point_centres_the_minimum(G):
+    W = _random_weights(G)
     q, z, s, _ = oracle.quantize(W, G)
     N, K = W.shape
     v = W.astype(np.float64).reshape(N, K // G, G)
@@ -130,11 +134,12 @@ def _half_ulp(a):
     return np.exp2(e - 11)
 
 
-def test_error_bound_on_non_degenerate_groups():
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_error_bound_on_non_degenerate_groups(G):
     """|v - W^| <= s/2 + max(0, (hi - lo) - 15 s) + ulp(W^)/2 whenever the zero
     point is not clamped (q cannot clamp at 0 then; at 15 the overshoot of the
     range beyond 15 s is the only extra error)."""
-    W = _random_weights()
+    W = _random_weights(G)
     q, z, s, _ = oracle.quantize(W, G)
     wh = oracle.dequant(q, z, s, G).astype(np.float64)
     N, K = W.shape
