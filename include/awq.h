@@ -6,8 +6,9 @@
  * README sections "Speed Benchmarks" and "Usage", step 3):
  *   weights are stored as 4-bit unsigned codes q with one fp16 scale s and one
  *   4-bit zero point z per (output channel, group of 128 input channels)
- *   ("--w_bit 4 --q_group_size 128"), each weight is w = (q - z) * s, and the
- *   layer runs as W4A16: fp16 activations times 4-bit weights, fp16 output.
+ *   ("--w_bit 4 --q_group_size 128"; Falcon-7B uses groups of 64, and groups
+ *   of 32 are taken too), each weight is w = (q - z) * s, and the layer runs
+ *   as W4A16: fp16 activations times 4-bit weights, fp16 output.
  *
  *   y[m][n] = sum_k x[m][k] * W^[n][k],   W^[n][k] = fp16_rne((q - z) * s)
  *
@@ -20,11 +21,15 @@
  *   qweight  uint32, (N/16)*(K/128) blocks of 16 x 16 words (K*N/2 bytes)
  *            Block (nb, kb) is 1 KiB, holds output channels n = 16*nb + r
  *            (r = 0..15) and input channels 128*kb .. 128*kb + 127. Word w of
- *            row r holds k = 128*kb + 8*w + i for i = 0..7: the code of even i
- *            at bits 4*(i/2) .. 4*(i/2)+3 and the code of odd i at bits
+ *            row r holds k = 128*kb + k0(w) + i for i = 0..7: the code of even
+ *            i at bits 4*(i/2) .. 4*(i/2)+3 and the code of odd i at bits
  *            16 + 4*(i/2) .. 16 + 4*(i/2)+3. So (word >> 4*j) & 0x000F000F
- *            holds the adjacent pair k = 8w + 2j, 8w + 2j + 1 as two 16-bit
- *            lanes. Blocks are grouped by 8 row blocks (128 output channels):
+ *            holds the adjacent pair k0 + 2j, k0 + 2j + 1 as two 16-bit lanes.
+ *            For group 128, k0(w) = 8*w. For group 64 or 32, with w = 4*t + j
+ *            (t, j = 0..3) and J = group/32, k0(w) = group*(j/J) + 8*(t*J +
+ *            j%J): the words with the same j hold whole groups (group j/J of
+ *            the block), and words 4t .. 4t+3 hold a piece of every group.
+ *            Blocks are grouped by 8 row blocks (128 output channels):
  *            group gi = nb/8 holds R = min(8, N/16 - 8*gi) row blocks and is
  *            stored k-block-major, so block (nb, kb) is block number
  *            8*gi*(K/128) + kb*R + nb%8, and the R blocks of one k-block of
@@ -45,7 +50,7 @@
  * Conventions for every entry point
  * ---------------------------------------------------------------------------
  *   Shapes     M >= 0 (M = 0 is a no-op), K > 0 and K % 128 == 0, N > 0 and
- *              N % 16 == 0, group == 128 (else AWQ_ERR_UNSUPPORTED).
+ *              N % 16 == 0, group 128, 64 or 32 (else AWQ_ERR_UNSUPPORTED).
  *   Pointers   device pointers unless stated; all non-null (x and y may be
  *              null when M == 0) and 16-byte aligned (AWQ_ERR_INVALID_ARG /
  *              AWQ_ERR_ALIGNMENT). Outputs may not overlap inputs.
@@ -82,7 +87,7 @@ typedef enum awq_status {
   AWQ_ERR_SHAPE = 2,       /* M < 0, K <= 0, N <= 0, K % 128, N % 16, K % group */
   AWQ_ERR_ALIGNMENT = 3,   /* a pointer that is not 16-byte aligned */
   AWQ_ERR_WORKSPACE = 4,   /* ws_bytes below awq_workspace_bytes(...) */
-  AWQ_ERR_UNSUPPORTED = 5, /* group != 128, M above an entry's limit, no sm_100 device */
+  AWQ_ERR_UNSUPPORTED = 5, /* group not 32, 64 or 128, M above an entry's limit, no sm_100 device */
   AWQ_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed */
   AWQ_ERR_TIMEOUT = 7,     /* device side: a bounded pipeline wait expired */
   AWQ_ERR_NONFINITE = 8    /* device side: awq_pack met an inf or NaN weight */

@@ -30,13 +30,13 @@ def host(t: torch.Tensor, np_dtype) -> np.ndarray:
     return t.cpu().numpy().view(np_dtype)
 
 
-def gpu_pack(W: np.ndarray, ws: torch.Tensor | None = None):
+def gpu_pack(W: np.ndarray, ws: torch.Tensor | None = None, group: int = G):
     """fp16 W [N][K] -> GPU packed (qweight int32, scales fp16, zeros uint8); checks the status word."""
     N, K = W.shape
     w = to_dev(W.view(np.uint16), torch.float16)
     if ws is None:
-        ws = awq.new_workspace(0, K, N, w.device)
-    qw, sc, ze = awq.awq_pack(w, ws)
+        ws = awq.new_workspace(0, K, N, w.device, group)
+    qw, sc, ze = awq.awq_pack(w, ws, group)
     st = awq.awq_get_status(ws)
     assert st == awq.AWQ_OK, awq.awq_status_string(st)
     return qw, sc, ze
@@ -83,7 +83,7 @@ def sample_rows(N: int, count: int, seed: int = 0) -> np.ndarray:
     return np.array(sorted(rows), dtype=np.int64)
 
 
-def oracle_rows(x: np.ndarray, qw, sc, ze, N: int, K: int, rows: np.ndarray):
+def oracle_rows(x: np.ndarray, qw, sc, ze, N: int, K: int, rows: np.ndarray, group: int = G):
     """Oracle y, B [M][len(rows)] at the given output channels."""
     M = x.shape[0]
     ms = np.repeat(np.arange(M), len(rows))
@@ -92,7 +92,7 @@ def oracle_rows(x: np.ndarray, qw, sc, ze, N: int, K: int, rows: np.ndarray):
     order = np.lexsort((ms, ns))
     y = np.empty(len(ms))
     b = np.empty(len(ms))
-    yo, bo = oracle.linear_entries(x, qw, sc, ze, N, K, ms[order], ns[order])
+    yo, bo = oracle.linear_entries(x, qw, sc, ze, N, K, ms[order], ns[order], group)
     y[order] = yo
     b[order] = bo
     return y.reshape(M, len(rows)), b.reshape(M, len(rows))

@@ -47,13 +47,15 @@ def test_status_strings():
 
 def test_packed_sizes():
     assert awq.awq_packed_size(4096, 4096) == (4096 * 4096 // 2, 4096 // 128 * 4096 * 2, 4096 // 128 * 4096 // 2)
+    for g in (64, 32):  # TinyChat README, Usage step 3: Falcon-7B uses groups of 64
+        assert awq.awq_packed_size(4096, 4096, g) == (4096 * 4096 // 2, 4096 // g * 4096 * 2, 4096 // g * 4096 // 2)
     assert awq.awq_packed_size(11008, 4096)[0] == 11008 * 4096 // 2
 
 
 @pytest.mark.parametrize("K,N,group,code", [
     (100, 16, 128, awq.AWQ_ERR_SHAPE), (128, 15, 128, awq.AWQ_ERR_SHAPE), (0, 16, 128, awq.AWQ_ERR_SHAPE),
     (128, 0, 128, awq.AWQ_ERR_SHAPE), (-128, 16, 128, awq.AWQ_ERR_SHAPE), (192, 16, 128, awq.AWQ_ERR_SHAPE),
-    (128, 16, 64, awq.AWQ_ERR_UNSUPPORTED), (128, 16, 32, awq.AWQ_ERR_UNSUPPORTED),
+    (128, 16, 256, awq.AWQ_ERR_UNSUPPORTED), (128, 16, 96, awq.AWQ_ERR_UNSUPPORTED), (128, 16, 16, awq.AWQ_ERR_UNSUPPORTED),
     (1 << 23, 16, 128, awq.AWQ_ERR_UNSUPPORTED),
 ])
 def test_packed_size_rejects(K, N, group, code):
@@ -84,7 +86,8 @@ def test_linear_argument_errors(fn):
     assert _linear(fn, M=-1) == awq.AWQ_ERR_SHAPE
     assert _linear(fn, K=4000) == awq.AWQ_ERR_SHAPE
     assert _linear(fn, N=4104) == awq.AWQ_ERR_SHAPE
-    assert _linear(fn, group=64) == awq.AWQ_ERR_UNSUPPORTED
+    assert _linear(fn, group=256) == awq.AWQ_ERR_UNSUPPORTED
+    assert _linear(fn, group=96) == awq.AWQ_ERR_UNSUPPORTED
     assert _linear(fn, x=None) == awq.AWQ_ERR_INVALID_ARG
     assert _linear(fn, y=None) == awq.AWQ_ERR_INVALID_ARG
     assert _linear(fn, ws=None) == awq.AWQ_ERR_INVALID_ARG

@@ -14,32 +14,32 @@ pytestmark = pytest.mark.gpu
 G = 128
 
 
-def _packed(N, K, tag, std=0.02):
+def _packed(N, K, tag, std=0.02, group=G):
     W = awq_synth.matrix_f16(awq_synth.key(0, 96, f"{tag}/W"), N, K, std)
-    dev = gpu_pack(W)
+    dev = gpu_pack(W, group=group)
     return W, dev, packed_to_host(*dev)
 
 
-def _run(fn, x, dev, N, M=None):
+def _run(fn, x, dev, N, M=None, group=G):
     xd = to_dev(x.view(np.uint16), torch.float16)
     M = x.shape[0]
     K = x.shape[1]
-    ws = awq.new_workspace(M, K, N, xd.device)
-    y = fn(xd, *dev, N, ws)
+    ws = awq.new_workspace(M, K, N, xd.device, group)
+    y = fn(xd, *dev, N, ws, group)
     st = awq.awq_get_status(ws)
     assert st == awq.AWQ_OK, awq.awq_status_string(st)
     return host(y, np.float16)
 
 
-def _check_against_oracle(y, x, hp, N, K, what):
+def _check_against_oracle(y, x, hp, N, K, what, group=G):
     """Every output when the oracle's work is small, else all tokens on
     sampled output channels (first and last row block plus random rows)."""
     M = x.shape[0]
     if M * N * K <= 2e8:
-        y_ref, b = oracle.linear(x, *hp, N, K)
+        y_ref, b = oracle.linear(x, *hp, N, K, group)
         return check_close(y, y_ref, b, what)
     rows = sample_rows(N, 64, seed=M)
-    y_ref, b = oracle_rows(x, *hp, N, K, rows)
+    y_ref, b = oracle_rows(x, *hp, N, K, rows, group)
     return check_close(y[:, rows], y_ref, b, what)
 
 
@@ -173,6 +173,45 @@ def test_gemv_multi_kblock_units(K, N, M):
     rows = np.array(sorted(rows), dtype=np.int64)
     y_ref, b = oracle_rows(x, *hp, N, K, rows)
     check_close(y[:, rows], y_ref, b, f"unit K={K} N={N} M={M}")
+
+
+# Group sizes 64 and 32 (TinyChat README, Usage step 3: Falcon-7B is quantized
+# with groups of 64). Small shapes (one-k-block units), a ragged one, and a
+# decode-sized layer whose units span 4 k-blocks, for the GEMV (M = 1, 5, 8,
+# 16, 32) and the GEMM.
+GROUP_SHAPES = [(256, 48), (1024, 592), (4096, 4096)]
+
+
+@pytest.mark.parametrize("group", [64, 32])
+@pytest.mark.parametrize("K,N", GROUP_SHAPES)
+@pytest.mark.parametrize("M", [1, 5, 8, 16, 32])
+def test_gemv_group_sizes(group, K, N, M):
+    W, dev, hp = _packed(N, K, f"g{group}/{K}x{N}", group=group)
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"g{group}/{K}x{N}/x{M}"), M, K, 1.0)
+    y = _run(awq.awq_w4a16_gemv, x, dev, N, group=group)
+    _check_against_oracle(y, x, hp, N, K, f"gemv g={group} M={M} K={K} N={N}", group)
+
+
+@pytest.mark.parametrize("group", [64, 32])
+@pytest.mark.parametrize("K,N", GROUP_SHAPES)
+@pytest.mark.parametrize("M", [7, 200, 513])
+def test_gemm_group_sizes(group, K, N, M):
+    W, dev, hp = _packed(N, K, f"g{group}/{K}x{N}", group=group)
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"g{group}m/{K}x{N}/x{M}"), M, K, 1.0)
+    y = _run(awq.awq_w4a16_gemm, x, dev, N, group=group)
+    _check_against_oracle(y, x, hp, N, K, f"gemm g={group} M={M} K={K} N={N}", group)
+
+
+@pytest.mark.parametrize("group", [64, 32])
+def test_group_sizes_multi_kblock_units(group):
+    K, N, M = 15616, 5168, 1   # 4 k-blocks per unit, K/128 = 122 (ragged), last group of 3 row blocks
+    W, dev, hp = _packed(N, K, f"g{group}unit", group=group)
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"g{group}unit/x"), M, K, 1.0)
+    y = _run(awq.awq_w4a16_gemv, x, dev, N, group=group)
+    rows = set(sample_rows(N, 64, seed=3).tolist()) | set(range(256)) | set(range(N - 256, N))
+    rows = np.array(sorted(rows), dtype=np.int64)
+    y_ref, b = oracle_rows(x, *hp, N, K, rows, group)
+    check_close(y[:, rows], y_ref, b, f"unit g={group}")
 
 
 PREFILL_CASES = [(l.name, M) for l in awq_synth.WORKLOADS["prefill"].layers for M in (512, 2048, 8192)]

@@ -38,10 +38,10 @@ def _adversarial(N=64, K=1024):
     return W.astype(np.float16)
 
 
-def _check_pack(W):
+def _check_pack(W, group=G):
     N, K = W.shape
-    qw, sc, ze = packed_to_host(*gpu_pack(W))
-    oq, osc, oze = oracle.quantize_pack(W)
+    qw, sc, ze = packed_to_host(*gpu_pack(W, group=group))
+    oq, osc, oze = oracle.quantize_pack(W, group)
     assert (qw == oq.reshape(qw.shape)).all(), "qweight differs"
     assert (sc.view(np.uint16) == osc.view(np.uint16)).all(), "scales differ"
     assert (ze == oze).all(), "zeros differ"
@@ -55,6 +55,24 @@ def test_pack_bit_exact_small(N, K):
 
 def test_pack_bit_exact_adversarial_groups():
     _check_pack(_adversarial())
+
+
+@pytest.mark.parametrize("group", [64, 32])
+@pytest.mark.parametrize("N,K", [(16, 128), (48, 384), (272, 640)])
+def test_pack_bit_exact_group_sizes(group, N, K):
+    W = awq_synth.matrix_f16(awq_synth.key(0, 97, f"pack{group}/{N}x{K}"), N, K, 0.02)
+    _check_pack(W, group)
+
+
+@pytest.mark.parametrize("group", [64, 32])
+def test_pack_and_dequant_bit_exact_adversarial_group_sizes(group):
+    W = _adversarial()
+    N, K = W.shape
+    _check_pack(W, group)
+    qw, sc, ze = gpu_pack(W, group=group)
+    wh = host(awq.awq_dequant(qw, sc, ze, K, N, group), np.float16)
+    q, z, s, _ = oracle.quantize(W, group)
+    assert (wh.view(np.uint16) == oracle.dequant(q, z, s, group).view(np.uint16)).all()
 
 
 def test_dequant_bit_exact():

@@ -86,6 +86,6 @@ def test_argument_errors():
     args = [x.data_ptr(), qw.data_ptr(), sc.data_ptr(), ze.data_ptr(), y.data_ptr()]
     assert L.awq_w4a16_gemv_no_alloc(*args, 33, 128, 16, 128, s) == awq.AWQ_ERR_UNSUPPORTED
     assert L.awq_w4a16_gemv_no_alloc(*args, 1, 100, 16, 128, s) == awq.AWQ_ERR_SHAPE
-    assert L.awq_w4a16_gemv_no_alloc(*args, 1, 128, 16, 64, s) == awq.AWQ_ERR_UNSUPPORTED
+    assert L.awq_w4a16_gemv_no_alloc(*args, 1, 128, 16, 96, s) == awq.AWQ_ERR_UNSUPPORTED
     assert L.awq_w4a16_gemv_no_alloc(None, *args[1:], 1, 128, 16, 128, s) == awq.AWQ_ERR_INVALID_ARG
     assert L.awq_w4a16_gemv_no_alloc(*args, 0, 128, 16, 128, s) == awq.AWQ_OK

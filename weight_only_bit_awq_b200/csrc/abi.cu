@@ -40,7 +40,7 @@ inline bool overlap(const void* a, size_t an, const void* b, size_t bn) {
 
 awq_status check_kn(int64_t K, int64_t N, int group) {
   if (K <= 0 || N <= 0) return AWQ_ERR_SHAPE;
-  if (group != 128) return AWQ_ERR_UNSUPPORTED;
+  if (group != 128 && group != 64 && group != 32) return AWQ_ERR_UNSUPPORTED;
   if (K % kKPerBlock != 0 || K % group != 0 || N % kRowsPerBlock != 0) return AWQ_ERR_SHAPE;
   if (K > kMaxK || N > kMaxN) return AWQ_ERR_UNSUPPORTED;
   return AWQ_OK;
@@ -121,7 +121,7 @@ int sm_count_or_default() {
 }
 
 awq_status gemv_impl(const LinearArgs& a, cudaStream_t stream) {
-  const GemvPlan p = plan_gemv(a.M, a.K, a.N, device_info().sm_count);
+  const GemvPlan p = plan_gemv(a.M, a.K, a.N, a.group, device_info().sm_count);
   cudaError_t e = launch_gemv(static_cast<const __half*>(a.x), static_cast<const uint32_t*>(a.qweight),
                               static_cast<const __half*>(a.scales), static_cast<const uint8_t*>(a.zeros),
                               static_cast<__half*>(a.y), a.M, a.K, a.N, a.workspace, p, stream);
@@ -131,7 +131,7 @@ awq_status gemv_impl(const LinearArgs& a, cudaStream_t stream) {
 awq_status gemm_impl(const LinearArgs& a, cudaStream_t stream) {
   cudaError_t e = launch_gemm(static_cast<const __half*>(a.x), static_cast<const uint32_t*>(a.qweight),
                               static_cast<const __half*>(a.scales), static_cast<const uint8_t*>(a.zeros),
-                              static_cast<__half*>(a.y), a.M, a.K, a.N, status_word(a.workspace), stream);
+                              static_cast<__half*>(a.y), a.M, a.K, a.N, a.group, status_word(a.workspace), stream);
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
@@ -155,7 +155,7 @@ size_t awq_workspace_bytes(int64_t M, int64_t K, int64_t N, int group) {
   if (M < 0 || check_kn(K, N, group) != AWQ_OK || M > kMaxM) return 0;
   size_t need = kWsHeaderBytes;
   if (M >= 1 && M <= AWQ_GEMV_MAX_M) {
-    const GemvPlan p = plan_gemv(M, K, N, sm_count_or_default());
+    const GemvPlan p = plan_gemv(M, K, N, group, sm_count_or_default());
     if (p.ws_bytes > need) need = p.ws_bytes;
   }
   return need;
@@ -182,7 +182,7 @@ awq_status awq_pack(const void* w, int64_t K, int64_t N, int group, void* qweigh
     return AWQ_ERR_INVALID_ARG;
   if (ws_bytes < kWsHeaderBytes) return AWQ_ERR_WORKSPACE;
   if ((st = check_device()) != AWQ_OK) return st;
-  cudaError_t e = launch_pack(static_cast<const __half*>(w), K, N, static_cast<uint32_t*>(qweight),
+  cudaError_t e = launch_pack(static_cast<const __half*>(w), K, N, group, static_cast<uint32_t*>(qweight),
                               static_cast<__half*>(scales), static_cast<uint8_t*>(zeros), status_word(workspace),
                               static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
@@ -200,7 +200,7 @@ awq_status awq_dequant(const void* qweight, const void* scales, const void* zero
     return AWQ_ERR_INVALID_ARG;
   if ((st = check_device()) != AWQ_OK) return st;
   cudaError_t e = launch_dequant(static_cast<const uint32_t*>(qweight), static_cast<const __half*>(scales),
-                                 static_cast<const uint8_t*>(zeros), K, N, static_cast<__half*>(w_out),
+                                 static_cast<const uint8_t*>(zeros), K, N, group, static_cast<__half*>(w_out),
                                  static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
@@ -244,7 +244,7 @@ int awq_linear_gemv_limit(void) { return g_gemv_limit; }
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group) {
   if (M <= 0 || M > kMaxM || check_kn(K, N, group) != AWQ_OK) return 0;
   if (M > g_gemv_limit) return 1;
-  return plan_gemv(M, K, N, sm_count_or_default()).has_split ? 2 : 1;
+  return plan_gemv(M, K, N, group, sm_count_or_default()).has_split ? 2 : 1;
 }
 
 awq_status awq_check_bounded_wait(void* workspace, size_t ws_bytes, uint32_t limit_us, void* stream) {
@@ -275,7 +275,7 @@ const char* awq_status_string(awq_status status) {
     case AWQ_ERR_SHAPE: return "AWQ_ERR_SHAPE: need M >= 0, K > 0, N > 0, K % 128 == 0, N % 16 == 0";
     case AWQ_ERR_ALIGNMENT: return "AWQ_ERR_ALIGNMENT: every pointer must be 16-byte aligned";
     case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE: workspace smaller than awq_workspace_bytes()";
-    case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED: group != 128, size above a limit, or no sm_100 device";
+    case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED: group not 32, 64 or 128, size above a limit, or no sm_100 device";
     case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: a CUDA call or kernel launch failed";
     case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT: a bounded wait on the device expired";
     case AWQ_ERR_NONFINITE: return "AWQ_ERR_NONFINITE: awq_pack met an inf or NaN weight";

@@ -58,6 +58,7 @@ const DeviceInfo& device_info();   // current device
 
 // GEMV launch plan (shared by awq_workspace_bytes and the launcher).
 struct GemvPlan {
+  int group;            // quantization group size (128, 64 or 32)
   int nt;               // token tiles of 8 (1, 2 or 4)
   int ku;               // k-blocks per streamed unit (1, 2 or 4)
   int stages;           // depth of the shared-memory ring
@@ -69,17 +70,29 @@ struct GemvPlan {
   size_t zero_bytes;    // bytes at the start of the workspace that must be zero at launch
   size_t ws_bytes;      // total workspace bytes
 };
-GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int sm_count);
+GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int group, int sm_count);
 
 // Launchers (argument checks are done by the ABI layer).
-cudaError_t launch_pack(const __half* w, int64_t K, int64_t N, uint32_t* qweight, __half* scales, uint8_t* zeros,
-                        uint32_t* status, cudaStream_t stream);
+cudaError_t launch_pack(const __half* w, int64_t K, int64_t N, int group, uint32_t* qweight, __half* scales,
+                        uint8_t* zeros, uint32_t* status, cudaStream_t stream);
 cudaError_t launch_dequant(const uint32_t* qweight, const __half* scales, const uint8_t* zeros, int64_t K,
-                           int64_t N, __half* w_out, cudaStream_t stream);
+                           int64_t N, int group, __half* w_out, cudaStream_t stream);
 cudaError_t launch_gemv(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
                         __half* y, int64_t M, int64_t K, int64_t N, void* workspace, const GemvPlan& plan,
                         cudaStream_t stream);
 cudaError_t launch_gemm(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
-                        __half* y, int64_t M, int64_t K, int64_t N, uint32_t* status, cudaStream_t stream);
+                        __half* y, int64_t M, int64_t K, int64_t N, int group, uint32_t* status,
+                        cudaStream_t stream);
+
+// Packed word order inside a row's 128-input block, for group size G (128, 64
+// or 32): word w = 4t + j holds the eight inputs from k0(w) = G (j / J) +
+// 8 (t J + j % J), J = G / 32 (for G = 128 simply 8w). The four words with the
+// same j hold whole groups, group j / J of the block.
+__host__ __device__ __forceinline__ constexpr int word_k0(int w, int G) {
+  return G * ((w & 3) / (G / 32)) + 8 * ((w >> 2) * (G / 32) + (w & 3) % (G / 32));
+}
+__host__ __device__ __forceinline__ constexpr int word_of_k(int k, int G) {
+  return 4 * (((k % G) / 8) / (G / 32)) + (k / G) * (G / 32) + ((k % G) / 8) % (G / 32);
+}
 
 }  // namespace awq

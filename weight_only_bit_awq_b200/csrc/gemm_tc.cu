@@ -43,6 +43,10 @@ constexpr int kXStages = 4;
 constexpr int kWStages = 2;
 constexpr int kQStages = 3;
 constexpr int kQBytes = 8 * 1024;
+// Behind a stage's codes: the tile's scale rows (up to 4 groups x 128 fp16)
+// and zero-point rows (up to 4 x 64 bytes) of that k-block.
+constexpr int kQScaleOff = kQBytes, kQZeroOff = kQScaleOff + 4 * 256;
+constexpr int kQStride = kQZeroOff + 4 * 64;
 constexpr int kWHalfBytes = kBM * 64 * 2;  // 16 KiB: 128 rows x 64 k
 constexpr int kWBytes = 2 * kWHalfBytes;
 constexpr int kWarpX = 0, kWarpMma = 1, kWarpQ = 2, kFirstDeqWarp = 3, kNumDeqWarps = 4;
@@ -61,7 +65,7 @@ struct Layout {
   static constexpr int kXOff = 0;
   static constexpr int kWOff = kXOff + kXStages * kXBytes;
   static constexpr int kQOff = kWOff + kWStages * kWBytes;
-  static constexpr int kBarOff = kQOff + kQStages * kQBytes;
+  static constexpr int kBarOff = kQOff + kQStages * kQStride;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1 KiB
@@ -79,7 +83,7 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// Eight codes of one word (k = 8w .. 8w+7) -> eight fp16 W^ = fp16_rne((q - z) s).
+// Eight codes of one word (inputs k0 .. k0+7) -> eight fp16 W^ = fp16_rne((q - z) s).
 // (word & 0x000F000F) | 0x64006400 = half2(1024 + q_even, 1024 + q_odd); the
 // 0x00F000F0 mask gives 1024 + 16 q. Subtracting 1024 + z (or scaling by 1/16
 // and subtracting 64 + z) is exact, and so the only rounding is that of the
@@ -95,7 +99,8 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, __half2 zlo, __half2 z
   return o;
 }
 
-template <int BN>
+// GS: group size (128, 64 or 32), kGPK = 128 / GS groups per k-block.
+template <int BN, int GS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
                 const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M,
@@ -123,7 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(bar(kBarWEmpty + i), 1);
     }
     for (int i = 0; i < kQStages; ++i) {
-      ptx::mbar_init(bar(kBarQFull + i), 1);
+      // the codes' byte count + 32 cp.async arrivals (scales, zeros)
+      ptx::mbar_init(bar(kBarQFull + i), 33);
       ptx::mbar_init(bar(kBarQEmpty + i), kDeqThreads);
     }
     ptx::mbar_init(bar(kBarAcc), 1);
@@ -161,23 +167,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kWarpQ) {
     // ---------------- packed-weight producer ----------------
-    if (lane == 0) {
-      // The R <= 8 row blocks of this tile's group are one contiguous run of
-      // R KiB per k-block in the packed layout: one 1-D bulk copy each.
-      const int64_t NB = N / kRowsPerBlock, gi = blockIdx.y;
-      const uint32_t qbytes = (uint32_t)(group_rows(gi, NB) * 1024);
-      int kb = 0;
-      for (; kb < KB; ++kb) {
-        const int s = kb % kQStages;
-        if (!wait_bar(bar(kBarQEmpty + s), ((kb / kQStages) & 1) ^ 1, abort_flag, status)) break;
-        ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qbytes);
-        ptx::bulk_g2s(sbase + L::kQOff + s * kQBytes, qweight + unit_first_block(gi, kb, KB, NB) * kWordsPerBlock,
-                      qbytes, bar(kBarQFull + s));
+    // The R <= 8 row blocks of this tile's group are one contiguous run of
+    // R KiB per k-block in the packed layout: one 1-D bulk copy each. The
+    // tile's scale and zero-point rows of the k-block follow by cp.async.
+    constexpr int kGPK = kKPerBlock / GS;
+    const int64_t NB = N / kRowsPerBlock, gi = blockIdx.y;
+    const uint32_t qbytes = (uint32_t)(group_rows(gi, NB) * 1024);
+    int kb = 0;
+    for (; kb < KB; ++kb) {
+      const int s = kb % kQStages;
+      bool ok = true;
+      if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((kb / kQStages) & 1) ^ 1, abort_flag, status);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const uint32_t st = sbase + L::kQOff + s * kQStride;
+      if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qbytes);
+      __syncwarp();
+      if (lane == 0)
+        ptx::bulk_g2s(st, qweight + unit_first_block(gi, kb, KB, NB) * kWordsPerBlock, qbytes, bar(kBarQFull + s));
+      for (int p = lane; p < kGPK * 16; p += 32) {  // kGPK rows of 128 scales: 16 B = 8 output channels
+        const int g = p >> 4, l = p & 15;
+        if (n0 + 8 * l < N)
+          ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
       }
-      if (kb < KB)
-        for (int j = (kb > kQStages ? kb - kQStages : 0); j < kb; ++j)
-          drain_bar(bar(kBarQFull + j % kQStages), (j / kQStages) & 1);
+      for (int p = lane; p < kGPK * 8; p += 32) {  // kGPK rows of 64 zero bytes: 8 B = 16 output channels
+        const int g = p >> 3, l = p & 7;
+        if (n0 + 16 * l < N)
+          ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l,
+                          zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
+      }
+      ptx::cp_async_arrive_noinc(bar(kBarQFull + s));
     }
+    if (kb < KB && lane == 0)
+      for (int j = (kb > kQStages ? kb - kQStages : 0); j < kb; ++j)
+        drain_bar(bar(kBarQFull + j % kQStages), (j / kQStages) & 1);
     __syncwarp();
   } else if (warp == kWarpMma) {
     // ---------------- MMA issuer ----------------
@@ -213,46 +235,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- dequantize, then epilogue ----------------
     const int row = threadIdx.x - kFirstDeqWarp * 32;  // 0..127, row & 31 == lane
-    const int n = n0 + row;
-    const bool valid = n < N;
     const int rot = (lane >> 1) & 3;  // chunk rotation: conflict-free shared loads and stores
+    constexpr int kGPK = kKPerBlock / GS;
     bool ok = true;
-    float s_next = 0.f;
-    uint32_t z_next = 0;
-    if (valid) {
-      s_next = __half2float(scales[n]);
-      z_next = (zeros[n >> 1] >> (4 * (n & 1))) & 0xF;
-    }
     for (int kb = 0; kb < KB; ++kb) {
-      const float s = s_next;
-      const uint32_t z = z_next;
-      if (valid && kb + 1 < KB) {
-        s_next = __half2float(scales[(int64_t)(kb + 1) * N + n]);
-        z_next = (zeros[(int64_t)(kb + 1) * (N / 2) + (n >> 1)] >> (4 * (n & 1))) & 0xF;
-      }
       const int qs = kb % kQStages;
       if (!(ok = wait_bar(bar(kBarQFull + qs), (kb / kQStages) & 1, abort_flag, status))) break;
-      const uint8_t* qrow = smem + L::kQOff + qs * kQBytes + (row >> 4) * 1024 + (row & 15) * 64;
+      const uint8_t* qst = smem + L::kQOff + qs * kQStride;
+      const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64;
       uint4 c[4];
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 3));
+      // fp16 bits of the scale and the zero point of this row, per group (rows
+      // past N read stale values: their outputs are never stored)
+      uint32_t s[kGPK], z[kGPK];
+#pragma unroll
+      for (int g = 0; g < kGPK; ++g) {
+        s[g] = reinterpret_cast<const uint16_t*>(qst + kQScaleOff + 256 * g)[row];
+        z[g] = (qst[kQZeroOff + 64 * g + (row >> 1)] >> (4 * (row & 1))) & 0xF;
+      }
       ptx::mbar_arrive(bar(kBarQEmpty + qs));
 
       const int ws = kb % kWStages;
       if (!(ok = wait_bar(bar(kBarWEmpty + ws), ((kb / kWStages) & 1) ^ 1, abort_flag, status))) break;
-      const __half2 s2 = __half2half2(__float2half_rn(s));
-      const __half2 zlo = __half2half2(__ushort_as_half((unsigned short)(0x6400u + z)));
-      const __half2 zhi = __half2half2(__float2half_rn(-64.0f - (float)z));
+      __half2 s2[kGPK], zlo[kGPK], zhi[kGPK];
+#pragma unroll
+      for (int g = 0; g < kGPK; ++g) {
+        // fp16 bit patterns: s itself, 1024 + z = 0x6400 + z, -(64 + z) = 0xD400 + 16 z
+        s2[g] = u2h(s[g] * 0x00010001u);
+        zlo[g] = u2h((0x6400u + z[g]) * 0x00010001u);
+        zhi[g] = u2h((0xD400u + (z[g] << 4)) * 0x00010001u);
+      }
       uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
-        const int cj = (jj + rot) & 3;  // which 32-k chunk of the block c[jj] holds
-        uint8_t* dst = wt + (cj >> 1) * kWHalfBytes;
+        const int cj = (jj + rot) & 3;  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
         const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
 #pragma unroll
         for (int ww = 0; ww < 4; ++ww) {
-          const int chunk = 4 * (cj & 1) + ww;  // 16-byte chunk (8 k) within the 64-k half
-          *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) = dequant_word(words[ww], zlo, zhi, s2);
+          // word 4 cj + ww holds inputs k0 .. k0 + 7 of group ww / (GS / 32)
+          // (word_k0 written out for this word: ww is a constant here)
+          constexpr int J = GS / 32;
+          const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
+          const int chunk = (k0 & 63) >> 3;  // 16-byte chunk (8 k) within the 64-k half
+          uint8_t* dst = wt + (k0 >> 6) * kWHalfBytes;
+          *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) = dequant_word(words[ww], zlo[g], zhi[g], s2[g]);
         }
       }
       ptx::fence_proxy_async_smem();
@@ -301,7 +328,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-template <int BN>
+template <int BN, int GS>
 cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
                       __half* y, int64_t M, int64_t K, int64_t N, uint32_t* status, cudaStream_t stream) {
   using L = Layout<BN>;
@@ -322,22 +349,34 @@ cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* sc
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
   if (!(attr_set >> dev & 1)) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
   }
   dim3 grid((unsigned)((M + BN - 1) / BN), (unsigned)((N + kBM - 1) / kBM));
-  gemm_kernel<BN><<<grid, kThreads, L::kAlloc, stream>>>(tx, qweight, scales, zeros, y, (int)M, (int)K, (int)N,
-                                                          status);
+  gemm_kernel<BN, GS><<<grid, kThreads, L::kAlloc, stream>>>(tx, qweight, scales, zeros, y, (int)M, (int)K, (int)N,
+                                                              status);
   return cudaGetLastError();
+}
+
+template <int GS>
+cudaError_t launch_gs(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
+                      __half* y, int64_t M, int64_t K, int64_t N, uint32_t* status, cudaStream_t stream) {
+  if (M > 128) return launch_bn<256, GS>(x, qweight, scales, zeros, y, M, K, N, status, stream);
+  return launch_bn<128, GS>(x, qweight, scales, zeros, y, M, K, N, status, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
-                        __half* y, int64_t M, int64_t K, int64_t N, uint32_t* status, cudaStream_t stream) {
-  if (M > 128) return launch_bn<256>(x, qweight, scales, zeros, y, M, K, N, status, stream);
-  return launch_bn<128>(x, qweight, scales, zeros, y, M, K, N, status, stream);
+                        __half* y, int64_t M, int64_t K, int64_t N, int group, uint32_t* status,
+                        cudaStream_t stream) {
+  switch (group) {
+    case 128: return launch_gs<128>(x, qweight, scales, zeros, y, M, K, N, status, stream);
+    case 64: return launch_gs<64>(x, qweight, scales, zeros, y, M, K, N, status, stream);
+    case 32: return launch_gs<32>(x, qweight, scales, zeros, y, M, K, N, status, stream);
+    default: return cudaErrorInvalidConfiguration;
+  }
 }
 
 }  // namespace awq

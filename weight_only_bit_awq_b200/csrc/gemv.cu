@@ -54,25 +54,27 @@ constexpr int kWarpXsum = 1 + kConsumers;  // per-k-block sums of x (M <= 8)
 constexpr int kThreads = (2 + kConsumers) * 32;
 constexpr int kMaxStages = 16;
 constexpr int kKbQBytes = kGroupBlocks * 1024;                    // codes of one k-block of a group
-constexpr int kKbScaleBytes = kGroupBlocks * kRowsPerBlock * 2;   // 256
-constexpr int kKbZeroBytes = kGroupBlocks * kRowsPerBlock / 2;    // 64
-constexpr int kKbXsBytes = 8 * 2 * 4;                             // 8 tokens x (C, X) fp32
+constexpr int kKbScaleBytes = kGroupBlocks * kRowsPerBlock * 2;   // 256: one row of scales (one group)
+constexpr int kKbZeroBytes = kGroupBlocks * kRowsPerBlock / 2;    // 64: one row of zero points
+constexpr int kKbXsBytes = 8 * 2 * 4;                             // 8 tokens x (C, X) fp32, per group
 constexpr int kXRowBytes = kKPerBlock * 2;                        // 256 bytes of x per token and k-block
 // Shared memory one CTA may use (two CTAs per SM share 228 KiB, minus the
 // 1 KiB per CTA the hardware reserves).
 constexpr int kSmemPerCta2 = 112 * 1024;
 constexpr int kSmemPerCta1 = 226 * 1024;
 
-// Byte offsets inside one ring stage for a unit of up to KU k-blocks and M
-// tokens (the same numbers on the host and in every thread).
+// Byte offsets inside one ring stage for a unit of up to KU k-blocks, M
+// tokens and groups of GS inputs (the same numbers on the host and in every
+// thread). Scales, zeros and x sums hold one row per group of the unit.
 struct Stage {
   int q, s, z, xs, x, bytes;
-  __host__ __device__ Stage(int KU, int M) {
+  __host__ __device__ Stage(int KU, int M, int GS) {
+    const int rows = KU * (kKPerBlock / GS);
     q = 0;
     s = q + KU * kKbQBytes;
-    z = s + KU * kKbScaleBytes;
-    xs = z + KU * kKbZeroBytes;
-    x = xs + KU * kKbXsBytes;
+    z = s + rows * kKbScaleBytes;
+    xs = z + rows * kKbZeroBytes;
+    x = xs + rows * kKbXsBytes;
     bytes = x + M * KU * kXRowBytes;  // every term is a multiple of 16
   }
 };
@@ -104,32 +106,46 @@ __device__ __forceinline__ void mma_16816_first(float (&d)[4], uint32_t a0, uint
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-// Independent accumulator chains per token tile: the 8 MMAs of a k-block are
-// spread over Chains accumulators so that consecutive MMAs do not wait on
-// each other's results.
-template <int NT>
-struct Chains {
-  static constexpr int value = NT == 1 ? 4 : 2;
+// Group size GS (128, 64 or 32) in the k-block of 128: the packed layout puts
+// the inputs of group j / J (J = GS / 32) into word 4t + j of every lane t, so
+// the MMAs of step j (one word per lane) see a single group. kGroupsPerKb
+// groups per k-block, each with its own scale and zero point.
+template <int GS>
+struct Grp {
+  static constexpr int J = GS / 32;              // MMA steps j per group
+  static constexpr int kPerKb = kKPerBlock / GS;  // groups per k-block
+  // byte offset, in a token's 128 x values of the k-block, of the 8 inputs in word 4t + j
+  __host__ __device__ static constexpr int x_off(int t, int j) { return 2 * word_k0(4 * t + j, GS); }
 };
 
-// acc[c][nt] = (q - z) * x over one k-block (split over the chains c), rows g
-// and g+8 (M > 8).
-template <int NT>
-__device__ __forceinline__ void block_mma(float (&acc)[Chains<NT>::value][NT][4], const uint4& wa4, const uint4& wb4,
-                                          uint32_t za, uint32_t zb, const uint4 (&xf)[NT][4]) {
-  constexpr int C = Chains<NT>::value;
+// Accumulators per token tile (M > 8): for GS = 128 the 8 MMAs of a k-block
+// are spread over two chains so that consecutive MMAs do not wait on each
+// other; for smaller groups there is one accumulator per group.
+template <int NT, int GS>
+struct Chains {
+  static constexpr int value = GS == 128 ? 2 : Grp<GS>::kPerKb;
+};
+
+// acc[c][nt] = (q - z) * x over one k-block, rows g and g+8 (M > 8); za, zb
+// are the zero points of the rows per group of the k-block.
+template <int NT, int GS>
+__device__ __forceinline__ void block_mma(float (&acc)[Chains<NT, GS>::value][NT][4], const uint4& wa4,
+                                          const uint4& wb4, const uint32_t (&za)[Grp<GS>::kPerKb],
+                                          const uint32_t (&zb)[Grp<GS>::kPerKb], const uint4 (&xf)[NT][4]) {
+  constexpr int C = Chains<NT, GS>::value, J = Grp<GS>::J;
   const uint32_t kMaskLo = 0x000F000Fu, kMaskHi = 0x00F000F0u, kMagic = 0x64006400u;
-  // Constants built from bit patterns (integer ops only, no conversions):
-  // fp16 1024 + z is 0x6400 + z, and -(64 + z) is 0xD400 + 16 z (z <= 15).
-  const __half2 zlo_a = u32_as_h2((0x6400u + za) * 0x00010001u);
-  const __half2 zlo_b = u32_as_h2((0x6400u + zb) * 0x00010001u);
-  const __half2 zhi_a = u32_as_h2((0xD400u + (za << 4)) * 0x00010001u);
-  const __half2 zhi_b = u32_as_h2((0xD400u + (zb << 4)) * 0x00010001u);
   const __half2 sixteenth = u32_as_h2(0x2C002C00u);  // 1/16
   const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
   const uint32_t wb[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
+    // Constants built from bit patterns (integer ops only, no conversions):
+    // fp16 1024 + z is 0x6400 + z, and -(64 + z) is 0xD400 + 16 z (z <= 15).
+    const int gk = j / J;
+    const __half2 zlo_a = u32_as_h2((0x6400u + za[gk]) * 0x00010001u);
+    const __half2 zlo_b = u32_as_h2((0x6400u + zb[gk]) * 0x00010001u);
+    const __half2 zhi_a = u32_as_h2((0xD400u + (za[gk] << 4)) * 0x00010001u);
+    const __half2 zhi_b = u32_as_h2((0xD400u + (zb[gk] << 4)) * 0x00010001u);
     uint32_t a = wa[j], b = wb[j];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -137,15 +153,17 @@ __device__ __forceinline__ void block_mma(float (&acc)[Chains<NT>::value][NT][4]
       const uint32_t a1 = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(b, kMaskLo, kMagic)), zlo_b));
       const uint32_t a2 = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(a, kMaskHi, kMagic)), sixteenth, zhi_a));
       const uint32_t a3 = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(b, kMaskHi, kMagic)), sixteenth, zhi_b));
-      const int idx = 2 * j + half;
+      const int step = 2 * j + half;
+      const int idx = GS == 128 ? step % C : gk;
+      const bool first = GS == 128 ? step < C : (j % J == 0 && half == 0);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const uint32_t b0 = half ? xf[nt][j].z : xf[nt][j].x;
         const uint32_t b1 = half ? xf[nt][j].w : xf[nt][j].y;
-        if (idx < C)
+        if (first)
           mma_16816_first(acc[idx][nt], a0, a1, a2, a3, b0, b1);
         else
-          mma_16816(acc[idx % C][nt], a0, a1, a2, a3, b0, b1);
+          mma_16816(acc[idx][nt], a0, a1, a2, a3, b0, b1);
       }
       a >>= 8;
       b >>= 8;
@@ -163,30 +181,40 @@ __device__ __forceinline__ float pos_half_bits_to_float(uint32_t h) {
 // M <= 8 (one token tile): the codes go into the MMA unchanged, as the fp16
 // values 1024 + q (pairs taken with the 0x000F000F mask, "lo" k) and
 // 1024 + 16 q (0x00F000F0 mask, "hi" k), in separate MMAs so that the two
-// offsets can be removed afterwards with per-k-block sums of x:
+// offsets can be removed afterwards with per-group sums of x:
 //   sum_k x (q - z) = acc_lo + acc_hi / 16 - (1024 X_lo + 64 X_hi) - z (X_lo + X_hi)
-// with X_lo, X_hi the sums of x over the lo and hi k of the k-block. This needs
-// 5 integer ops per 8 weights and no fp16 arithmetic. acc[0..1] are lo chains,
-// acc[2..3] hi chains.
-__device__ __forceinline__ void block_mma_lohi(float (&acc)[4][4], const uint4& wa4, const uint4& wb4,
+// with X_lo, X_hi the sums of x over the lo and hi k of the group. This needs
+// 5 integer ops per 8 weights and no fp16 arithmetic. LoHi<GS>::kAcc
+// accumulators: lo ones first, then hi ones; for GS = 128 two chains of each,
+// else one of each per group.
+template <int GS>
+struct LoHi {
+  static constexpr int kLo = GS == 128 ? 2 : Grp<GS>::kPerKb;
+  static constexpr int kAcc = 2 * kLo;
+};
+template <int GS>
+__device__ __forceinline__ void block_mma_lohi(float (&acc)[LoHi<GS>::kAcc][4], const uint4& wa4, const uint4& wb4,
                                                const uint4 (&xf)[4]) {
+  constexpr int kLo = LoHi<GS>::kLo, J = Grp<GS>::J;
   const uint32_t kMaskLo = 0x000F000Fu, kMaskHi = 0x00F000F0u, kMagic = 0x64006400u;
   const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
   const uint32_t wb[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t a = wa[j], b = wb[j], a8 = wa[j] >> 8, b8 = wb[j] >> 8;
-    // slots (2t, 2t+1) <- k = 8j + 0, 1 (lo) / 2, 3 (hi); slots (2t+8, 2t+9) <- 4, 5 / 6, 7
+    // slots (2t, 2t+1) <- k0 + 0, 1 (lo) / 2, 3 (hi); slots (2t+8, 2t+9) <- k0 + 4, 5 / 6, 7
     const uint32_t l0 = lop3_and_or(a, kMaskLo, kMagic), l1 = lop3_and_or(b, kMaskLo, kMagic);
     const uint32_t l2 = lop3_and_or(a8, kMaskLo, kMagic), l3 = lop3_and_or(b8, kMaskLo, kMagic);
     const uint32_t h0 = lop3_and_or(a, kMaskHi, kMagic), h1 = lop3_and_or(b, kMaskHi, kMagic);
     const uint32_t h2 = lop3_and_or(a8, kMaskHi, kMagic), h3 = lop3_and_or(b8, kMaskHi, kMagic);
-    if (j < 2) {
-      mma_16816_first(acc[j], l0, l1, l2, l3, xf[j].x, xf[j].z);
-      mma_16816_first(acc[2 + j], h0, h1, h2, h3, xf[j].y, xf[j].w);
+    const int idx = GS == 128 ? (j & 1) : j / J;
+    const bool first = GS == 128 ? j < 2 : j % J == 0;
+    if (first) {
+      mma_16816_first(acc[idx], l0, l1, l2, l3, xf[j].x, xf[j].z);
+      mma_16816_first(acc[kLo + idx], h0, h1, h2, h3, xf[j].y, xf[j].w);
     } else {
-      mma_16816(acc[j & 1], l0, l1, l2, l3, xf[j].x, xf[j].z);
-      mma_16816(acc[2 + (j & 1)], h0, h1, h2, h3, xf[j].y, xf[j].w);
+      mma_16816(acc[idx], l0, l1, l2, l3, xf[j].x, xf[j].z);
+      mma_16816(acc[kLo + idx], h0, h1, h2, h3, xf[j].y, xf[j].w);
     }
   }
 }
@@ -207,15 +235,17 @@ struct Range {
   __host__ __device__ __forceinline__ int64_t cta_of(int64_t u) const { return ((u + 1) * P - 1) / U; }
 };
 
-// kM1: M == 1 (NT == 1), where only the epilogue slots of token 0 are computed.
-template <int NT, int KU, bool kM1>
+// kM1: M == 1 (NT == 1), where only the epilogue slots of token 0 are
+// computed. GS: group size (128, 64 or 32).
+template <int NT, int KU, bool kM1, int GS>
 __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
     gemv_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight, const __half* __restrict__ scales,
                 const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M, int K, int N, int NS,
                 float* __restrict__ partial, uint32_t* status) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr bool kLoHi = NT == 1;
-  const Stage L(KU, M);
+  constexpr int kGPK = Grp<GS>::kPerKb;  // groups per k-block
+  const Stage L(KU, M, GS);
   const uint32_t sbase = ptx::smem_u32(smem);
   const uint32_t bar0 = sbase + NS * L.bytes;
   auto full = [&](int s) -> uint32_t { return bar0 + 8 * s; };
@@ -259,13 +289,13 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       if (lane == 0)
         ptx::bulk_g2s(st + L.q, qweight + unit_first_block(cgi, kb0, rg.KB, rg.NB) * kWordsPerBlock,
                       (uint32_t)(ku * R * 1024), full(s));
-      const __half* srow = scales + kb0 * N + kGroupBlocks * kRowsPerBlock * cgi;
-      for (int p = lane; p < ku * 16; p += 32) {  // ku rows of 32 R bytes
+      const __half* srow = scales + kb0 * kGPK * N + kGroupBlocks * kRowsPerBlock * cgi;
+      for (int p = lane; p < ku * kGPK * 16; p += 32) {  // ku * kGPK rows of 32 R bytes
         const int j = p >> 4, l = p & 15;
         if (l < 2 * R) ptx::cp_async_16(st + L.s + j * kKbScaleBytes + 16 * l, srow + (int64_t)j * N + 8 * l);
       }
-      const uint8_t* zrow = zeros + kb0 * (N / 2) + 64 * cgi;
-      for (int p = lane; p < ku * 8; p += 32) {  // ku rows of 8 R bytes
+      const uint8_t* zrow = zeros + kb0 * kGPK * (N / 2) + 64 * cgi;
+      for (int p = lane; p < ku * kGPK * 8; p += 32) {  // ku * kGPK rows of 8 R bytes
         const int j = p >> 3, l = p & 7;
         if (l < R) ptx::cp_async_8(st + L.z + j * kKbZeroBytes + 8 * l, zrow + (int64_t)j * (N / 2) + 8 * l);
       }
@@ -317,7 +347,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
     // ------------------------------ x sums (M <= 8) ------------------------------
     // Per k-block j of the unit, lane (m, t4) = (lane / 4, lane % 4) adds token
     // m's x over k = 32 t4 .. 32 t4 + 31 into lo (k % 8 in {0, 1, 4, 5}) and hi
-    // (k % 8 in {2, 3, 6, 7}) fp32 sums.
+    // (k % 8 in {2, 3, 6, 7}) fp32 sums, then the lanes of one group (all four,
+    // two or one) add theirs.
     if (kLoHi) {
       const int m = lane >> 2, t4 = lane & 3;
       int jj = (int)(u0 % rg.UPG), s = 0, ph = 0;
@@ -339,12 +370,14 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
               hi += (p1.x + p1.y) + (p3.x + p3.y);
             }
           }
-          lo += __shfl_xor_sync(0xffffffffu, lo, 1);
-          hi += __shfl_xor_sync(0xffffffffu, hi, 1);
-          lo += __shfl_xor_sync(0xffffffffu, lo, 2);
-          hi += __shfl_xor_sync(0xffffffffu, hi, 2);
-          if (t4 == 0 && m < M) {
-            float* xs = reinterpret_cast<float*>(smem + s * L.bytes + L.xs + j * kKbXsBytes);
+#pragma unroll
+          for (int off = 1; off < GS / 32; off <<= 1) {
+            lo += __shfl_xor_sync(0xffffffffu, lo, off);
+            hi += __shfl_xor_sync(0xffffffffu, hi, off);
+          }
+          if (t4 % (GS / 32) == 0 && m < M) {
+            const int gk = t4 / (GS / 32);
+            float* xs = reinterpret_cast<float*>(smem + s * L.bytes + L.xs + (j * kGPK + gk) * kKbXsBytes);
             xs[2 * m] = 1024.f * lo + 64.f * hi;
             xs[2 * m + 1] = lo + hi;
           }
@@ -409,65 +442,83 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
   // what the epilogue needs besides the MMA results; kb_finish adds the
   // k-block to yacc. (Finishing a k-block only after the next one's MMAs were
   // issued measured no faster on B200.)
-  constexpr int kC = Chains<NT>::value;
-  using Acc = std::conditional_t<kLoHi, float[4][4], float[kC][NT][4]>;
+  constexpr int kC = Chains<NT, GS>::value;
+  using Acc = std::conditional_t<kLoHi, float[LoHi<GS>::kAcc][4], float[kC][NT][4]>;
   struct KState {
-    float s[2];     // scales of rows g, g + 8
-    float corr[4];  // lo/hi path: s (C + z X) of slot cc (rows g / g+8, tokens 2t / 2t+1)
+    float s[kGPK][2];     // scales of rows g, g + 8 per group of the k-block
+    float corr[kGPK][4];  // lo/hi path: s (C + z X) of slot cc (rows g / g+8, tokens 2t / 2t+1)
   };
   auto kb_issue = [&](const uint8_t* st, int j, int R, Acc& acc, KState& ks) {
     const uint8_t* blk = st + L.q + (j * R + cw) * 1024;
     const uint4 wa = *reinterpret_cast<const uint4*>(blk + g * 64 + 16 * t);
     const uint4 wb = *reinterpret_cast<const uint4*>(blk + (g + 8) * 64 + 16 * t);
-    const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + L.s + j * kKbScaleBytes) + cw * kRowsPerBlock;
-    ks.s[0] = pos_half_bits_to_float(sc[g]);
-    ks.s[1] = pos_half_bits_to_float(sc[g + 8]);
-    const uint8_t* zr = st + L.z + j * kKbZeroBytes + cw * (kRowsPerBlock / 2);
-    const uint32_t za = (zr[g >> 1] >> (4 * (g & 1))) & 0xF;
-    const uint32_t zb = (zr[(g + 8) >> 1] >> (4 * (g & 1))) & 0xF;
+    uint32_t za[kGPK], zb[kGPK];
+#pragma unroll
+    for (int gk = 0; gk < kGPK; ++gk) {
+      const uint16_t* sc =
+          reinterpret_cast<const uint16_t*>(st + L.s + (j * kGPK + gk) * kKbScaleBytes) + cw * kRowsPerBlock;
+      ks.s[gk][0] = pos_half_bits_to_float(sc[g]);
+      ks.s[gk][1] = pos_half_bits_to_float(sc[g + 8]);
+      const uint8_t* zr = st + L.z + (j * kGPK + gk) * kKbZeroBytes + cw * (kRowsPerBlock / 2);
+      za[gk] = (zr[g >> 1] >> (4 * (g & 1))) & 0xF;
+      zb[gk] = (zr[(g + 8) >> 1] >> (4 * (g & 1))) & 0xF;
+    }
+    // B fragment q of lane t: the token's 8 inputs in word 4t + q
     uint4 xf[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int m = 8 * nt + g;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        xf[nt][q] = m < M ? *reinterpret_cast<const uint4*>(st + L.x + (m * KU + j) * kXRowBytes + 64 * t + 16 * q)
+        xf[nt][q] = m < M ? *reinterpret_cast<const uint4*>(st + L.x + (m * KU + j) * kXRowBytes + Grp<GS>::x_off(t, q))
                           : make_uint4(0, 0, 0, 0);
     }
     if constexpr (kLoHi) {
-      block_mma_lohi(acc, wa, wb, xf[0]);
-      // C and X of tokens 2t and 2t + 1
-      const float4 cx = *reinterpret_cast<const float4*>(st + L.xs + j * kKbXsBytes + 16 * t);
-      const float zf[2] = {__uint_as_float(0x4B000000u | za) - 8388608.f,  // exact (float)z
-                           __uint_as_float(0x4B000000u | zb) - 8388608.f};
+      block_mma_lohi<GS>(acc, wa, wb, xf[0]);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        if (kM1 && (cc & 1)) continue;  // slots of token 1
-        const float Cm = (cc & 1) ? cx.z : cx.x, Xm = (cc & 1) ? cx.w : cx.y;
-        ks.corr[cc] = ks.s[cc >> 1] * fmaf(zf[cc >> 1], Xm, Cm);
+      for (int gk = 0; gk < kGPK; ++gk) {
+        // C and X of tokens 2t and 2t + 1 over group gk
+        const float4 cx = *reinterpret_cast<const float4*>(st + L.xs + (j * kGPK + gk) * kKbXsBytes + 16 * t);
+        const float zf[2] = {__uint_as_float(0x4B000000u | za[gk]) - 8388608.f,  // exact (float)z
+                             __uint_as_float(0x4B000000u | zb[gk]) - 8388608.f};
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          if (kM1 && (cc & 1)) continue;  // slots of token 1
+          const float Cm = (cc & 1) ? cx.z : cx.x, Xm = (cc & 1) ? cx.w : cx.y;
+          ks.corr[gk][cc] = ks.s[gk][cc >> 1] * fmaf(zf[cc >> 1], Xm, Cm);
+        }
       }
     } else {
-      block_mma<NT>(acc, wa, wb, za, zb, xf);
+      block_mma<NT, GS>(acc, wa, wb, za, zb, xf);
     }
   };
   auto kb_finish = [&](const Acc& acc, const KState& ks) {
     if constexpr (kLoHi) {
-      // y += s (acc_lo + acc_hi / 16) - s (C + z X)
+      // y += s (acc_lo + acc_hi / 16) - s (C + z X), per group
+      constexpr int kLo = LoHi<GS>::kLo;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        if (kM1 && (cc & 1)) continue;
-        const float lo = acc[0][cc] + acc[1][cc], hi = acc[2][cc] + acc[3][cc];
-        yacc[0][cc] = fmaf(ks.s[cc >> 1], fmaf(hi, 0.0625f, lo), yacc[0][cc]) - ks.corr[cc];
-      }
+      for (int gk = 0; gk < kGPK; ++gk)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          if (kM1 && (cc & 1)) continue;
+          const float lo = GS == 128 ? acc[0][cc] + acc[1][cc] : acc[gk][cc];
+          const float hi = GS == 128 ? acc[2][cc] + acc[3][cc] : acc[kLo + gk][cc];
+          yacc[0][cc] = fmaf(ks.s[gk][cc >> 1], fmaf(hi, 0.0625f, lo), yacc[0][cc]) - ks.corr[gk][cc];
+        }
     } else {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-          float v = acc[0][nt][cc];
+          if (GS == 128) {
+            float v = acc[0][nt][cc];
 #pragma unroll
-          for (int ch = 1; ch < kC; ++ch) v += acc[ch][nt][cc];
-          yacc[nt][cc] = fmaf(ks.s[cc >> 1], v, yacc[nt][cc]);
+            for (int ch = 1; ch < kC; ++ch) v += acc[ch][nt][cc];
+            yacc[nt][cc] = fmaf(ks.s[0][cc >> 1], v, yacc[nt][cc]);
+          } else {
+#pragma unroll
+            for (int gk = 0; gk < kGPK; ++gk) yacc[nt][cc] = fmaf(ks.s[gk][cc >> 1], acc[gk][nt][cc], yacc[nt][cc]);
+          }
         }
     }
   };
@@ -505,8 +556,11 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       const int64_t kb0 = (int64_t)jj * KU;
       const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
       if (ku == KU) {
-#pragma unroll 2
-        for (int j = 0; j < KU; ++j) kblock(st, j, R);  // no guard: pairs of k-blocks can interleave
+        // no guard: for one token tile pairs of k-blocks can interleave (more
+        // token tiles would run out of registers)
+        constexpr int kUnroll = NT == 1 ? 2 : 1;
+#pragma unroll kUnroll
+        for (int j = 0; j < KU; ++j) kblock(st, j, R);
       } else {
 #pragma unroll 1
         for (int j = 0; j < ku; ++j) kblock(st, j, R);
@@ -556,14 +610,14 @@ __global__ void __launch_bounds__(128) gemv_fixup_kernel(const float* __restrict
   y[(int64_t)m * N + gi * kGroupBlocks * kRowsPerBlock + threadIdx.x] = __float2half_rn(v);
 }
 
-template <int NT, int KU, bool kM1>
+template <int NT, int KU, bool kM1, int GS>
 cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros, __half* y,
                      int M, int K, int N, void* workspace, const GemvPlan& p, cudaStream_t stream) {
   static uint64_t attr_set = 0;  // one bit per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
   if (!(attr_set >> dev & 1)) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, KU, kM1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, KU, kM1, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          NT == 4 ? kSmemPerCta1 : kSmemPerCta2);
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
@@ -581,7 +635,7 @@ cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* sca
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<NT, KU, kM1>, x, qweight, scales, zeros, y, M, K, N, p.stages,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<NT, KU, kM1, GS>, x, qweight, scales, zeros, y, M, K, N, p.stages,
                                      partial, status);
   if (e != cudaSuccess || !p.has_split) return e;
   cudaLaunchConfig_t fcfg = cfg;
@@ -591,13 +645,26 @@ cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* sca
   return cudaLaunchKernelEx(&fcfg, gemv_fixup_kernel, (const float*)partial, y, M, K, N, p.ku, p.ctas);
 }
 
-template <int NT, bool kM1>
+template <int NT, bool kM1, int GS>
 cudaError_t launch_nt(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
                       __half* y, int M, int K, int N, void* workspace, const GemvPlan& p, cudaStream_t stream) {
   switch (p.ku) {
-    case 1: return launch_t<NT, 1, kM1>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
-    case 2: return launch_t<NT, 2, kM1>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
-    case 4: return launch_t<NT, 4, kM1>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    case 1: return launch_t<NT, 1, kM1, GS>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    case 2: return launch_t<NT, 2, kM1, GS>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    case 4: return launch_t<NT, 4, kM1, GS>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    default: return cudaErrorInvalidConfiguration;
+  }
+}
+
+template <int GS>
+cudaError_t launch_g(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
+                     __half* y, int m, int k, int n, void* workspace, const GemvPlan& p, cudaStream_t stream) {
+  switch (p.nt) {
+    case 1:
+      return m == 1 ? launch_nt<1, true, GS>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream)
+                    : launch_nt<1, false, GS>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
+    case 2: return launch_nt<2, false, GS>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
+    case 4: return launch_nt<4, false, GS>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
     default: return cudaErrorInvalidConfiguration;
   }
 }
@@ -611,8 +678,9 @@ cudaError_t launch_nt(const __half* x, const uint32_t* qweight, const __half* sc
 // than four 8 KiB ones.
 constexpr int kMinStages = 3;
 
-GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int sm_count) {
+GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int group, int sm_count) {
   GemvPlan p{};
+  p.group = group;
   p.nt = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
   const int64_t NB = N / kRowsPerBlock, KB = K / kKPerBlock;
   p.groups = (int)((NB + kGroupBlocks - 1) / kGroupBlocks);
@@ -621,7 +689,7 @@ GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int sm_count) {
   const int64_t Mi = M < 1 ? 1 : M;
   for (int ku : {4, 2, 1}) {
     const int64_t U = p.groups * ((KB + ku - 1) / ku);
-    const int stage = Stage(ku, (int)Mi).bytes;
+    const int stage = Stage(ku, (int)Mi, group).bytes;
     int stages = budget / stage;
     if (stages > kMaxStages) stages = kMaxStages;
     const bool last = ku == 1;
@@ -645,12 +713,10 @@ cudaError_t launch_gemv(const __half* x, const uint32_t* qweight, const __half* 
                         __half* y, int64_t M, int64_t K, int64_t N, void* workspace, const GemvPlan& p,
                         cudaStream_t stream) {
   const int m = (int)M, k = (int)K, n = (int)N;
-  switch (p.nt) {
-    case 1:
-      return m == 1 ? launch_nt<1, true>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream)
-                    : launch_nt<1, false>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
-    case 2: return launch_nt<2, false>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
-    case 4: return launch_nt<4, false>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
+  switch (p.group) {
+    case 128: return launch_g<128>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
+    case 64: return launch_g<64>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
+    case 32: return launch_g<32>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
     default: return cudaErrorInvalidConfiguration;
   }
 }

@@ -60,7 +60,7 @@ extern "C" awq_status awq_w4a16_gemv_no_alloc(const void* x, const void* qweight
                                               int group, void* stream) {
   using namespace awq;
   if (M < 0 || K <= 0 || N <= 0) return AWQ_ERR_SHAPE;
-  if (group != 128) return AWQ_ERR_UNSUPPORTED;
+  if (group != 128 && group != 64 && group != 32) return AWQ_ERR_UNSUPPORTED;
   if (K % kKPerBlock != 0 || N % kRowsPerBlock != 0) return AWQ_ERR_SHAPE;
   if (M > AWQ_GEMV_MAX_M) return AWQ_ERR_UNSUPPORTED;
   if ((M > 0 && (!x || !y)) || !qweight || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
@@ -75,7 +75,7 @@ extern "C" awq_status awq_w4a16_gemv_no_alloc(const void* x, const void* qweight
   void* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return AWQ_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const GemvPlan p = plan_gemv(M, K, N, d.sm_count);
+  const GemvPlan p = plan_gemv(M, K, N, group, d.sm_count);
   // The status word must start at zero; the partial sums are always written
   // before they are read.
   if (cudaMemsetAsync(scratch, 0, p.zero_bytes, s) != cudaSuccess) return AWQ_ERR_CUDA;

@@ -2,7 +2,8 @@
 //
 // TinyChat README, Usage step 3 ("--w_bit 4 --q_group_size 128 ...
 // --q_backend real"): fp16 weights become 4-bit codes with one fp16 scale and
-// one 4-bit zero point per (output channel, group of 128 input channels).
+// one 4-bit zero point per (output channel, group of 128 input channels);
+// Falcon-7B uses groups of 64 (same step), so G = 64 and 32 are taken too.
 // The arithmetic is asymmetric min-max (the pages print no formula; this is
 // its plainest reading), done in fp64 against the stored fp16 scale so that
 // the result is reproducible bit for bit:
@@ -25,17 +26,21 @@ __device__ __forceinline__ __half f64_to_f16_rn(double v) {
 __device__ __forceinline__ int nibble_shift(int i) { return (i & 1) ? 16 + 4 * (i >> 1) : 4 * (i >> 1); }
 
 // One CTA = one packed block (16 output channels x 128 input channels);
-// warp r quantizes row 16*nb + r, lane l owns k = 4l .. 4l+3 of the group.
-__global__ void __launch_bounds__(512) pack_kernel(const __half* __restrict__ w, int64_t K, int64_t N,
+// warp r quantizes row 16*nb + r, lane l owns k = 4l .. 4l+3 of the block, and
+// the G/4 lanes of one group (G = 128, 64 or 32) reduce its min and max.
+__global__ void __launch_bounds__(512) pack_kernel(const __half* __restrict__ w, int64_t K, int64_t N, int G,
                                                    uint32_t* __restrict__ qweight, __half* __restrict__ scales,
                                                    uint8_t* __restrict__ zeros, uint32_t* status) {
-  __shared__ uint8_t zbuf[kRowsPerBlock];
+  __shared__ uint8_t zbuf[kRowsPerBlock][kKPerBlock / 32];
   const int64_t nb = blockIdx.x;
   const int kb = blockIdx.y;
   const int r = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t KB = K / kKPerBlock;
   const int64_t n = nb * kRowsPerBlock + r;
+  const int gpk = kKPerBlock / G;        // groups per block
+  const int lanes = G / 4;               // lanes per group
+  const int gk = lane / lanes;           // this lane's group in the block
 
   const uint2 raw = *reinterpret_cast<const uint2*>(w + n * K + (int64_t)kb * kKPerBlock + 4 * lane);
   const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
@@ -50,12 +55,13 @@ __global__ void __launch_bounds__(512) pack_kernel(const __half* __restrict__ w,
     lo = fminf(lo, f[j]);
     hi = fmaxf(hi, f[j]);
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {  // fp16 values are exact in fp32
+  for (int off = lanes / 2; off > 0; off >>= 1) {  // fp16 values are exact in fp32
     lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
     hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
   }
-  const bool group_finite = __all_sync(0xffffffffu, finite);
+  const uint32_t finite_lanes = __ballot_sync(0xffffffffu, finite);
+  const uint32_t group_lanes = (lanes == 32 ? 0xffffffffu : ((1u << lanes) - 1u)) << (gk * lanes);
+  const bool group_finite = (finite_lanes & group_lanes) == group_lanes;
 
   uint32_t part = 0;
   uint8_t zq = 0;
@@ -75,30 +81,34 @@ __global__ void __launch_bounds__(512) pack_kernel(const __half* __restrict__ w,
       const int i = 4 * (lane & 1) + j;  // position of this k inside its 8-k word
       part |= (uint32_t)q << nibble_shift(i);
     }
-  } else if (lane == 0) {
+  } else if (lane % lanes == 0) {
     record_status(status, AWQ_ERR_NONFINITE);
   }
+  // lanes 2m, 2m+1 hold inputs 8m .. 8m+7, the word word_of_k(8m) of the row
   const uint32_t word = part | __shfl_xor_sync(0xffffffffu, part, 1);
   if ((lane & 1) == 0) {
-    qweight[(block_index(nb, kb, KB, N / kRowsPerBlock) * kRowsPerBlock + r) * kWordsPerRow + (lane >> 1)] = word;
+    qweight[(block_index(nb, kb, KB, N / kRowsPerBlock) * kRowsPerBlock + r) * kWordsPerRow +
+            word_of_k(4 * lane, G)] = word;
   }
-  if (lane == 0) {
-    scales[(int64_t)kb * N + n] = s16;
-    zbuf[r] = zq;
+  if (lane % lanes == 0) {
+    scales[((int64_t)kb * gpk + gk) * N + n] = s16;
+    zbuf[r][gk] = zq;
   }
   __syncthreads();
-  if (threadIdx.x < kRowsPerBlock / 2) {
-    const int j = threadIdx.x;
-    zeros[(int64_t)kb * (N / 2) + nb * (kRowsPerBlock / 2) + j] = (uint8_t)(zbuf[2 * j] | (zbuf[2 * j + 1] << 4));
+  if (threadIdx.x < gpk * (kRowsPerBlock / 2)) {
+    const int g = threadIdx.x / (kRowsPerBlock / 2), j = threadIdx.x % (kRowsPerBlock / 2);
+    zeros[((int64_t)kb * gpk + g) * (N / 2) + nb * (kRowsPerBlock / 2) + j] =
+        (uint8_t)(zbuf[2 * j][g] | (zbuf[2 * j + 1][g] << 4));
   }
 }
 
-// One CTA = one packed block; thread t expands word t (row t/16, 8 k values)
-// into eight fp16 weights W^ = fp16_rne((q - z) * s). (q - z) * s is exact in
-// fp32 (at most 4 + 11 significant bits), so one rounding to fp16 remains.
+// One CTA = one packed block; thread t expands word t (row t/16, the 8 inputs
+// from word_k0) into eight fp16 weights W^ = fp16_rne((q - z) * s). (q - z) * s
+// is exact in fp32 (at most 4 + 11 significant bits), so one rounding to fp16
+// remains.
 __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict__ qweight,
                                                       const __half* __restrict__ scales,
-                                                      const uint8_t* __restrict__ zeros, int64_t K, int64_t N,
+                                                      const uint8_t* __restrict__ zeros, int64_t K, int64_t N, int G,
                                                       __half* __restrict__ w_out) {
   const int64_t nb = blockIdx.x;
   const int kb = blockIdx.y;
@@ -106,31 +116,33 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
   const int r = t / kWordsPerRow, wi = t % kWordsPerRow;
   const int64_t KB = K / kKPerBlock;
   const int64_t n = nb * kRowsPerBlock + r;
+  const int k0 = word_k0(wi, G);
+  const int64_t grow = (int64_t)kb * (kKPerBlock / G) + k0 / G;  // row of the scale / zero tables
   const uint32_t word = qweight[block_index(nb, kb, KB, N / kRowsPerBlock) * kWordsPerBlock + t];
-  const float s = __half2float(scales[(int64_t)kb * N + n]);
-  const int z = (zeros[(int64_t)kb * (N / 2) + (n >> 1)] >> (4 * (n & 1))) & 0xF;
+  const float s = __half2float(scales[grow * N + n]);
+  const int z = (zeros[grow * (N / 2) + (n >> 1)] >> (4 * (n & 1))) & 0xF;
   __align__(16) __half out[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int q = (word >> nibble_shift(i)) & 0xF;
     out[i] = __float2half_rn((float)(q - z) * s);
   }
-  *reinterpret_cast<uint4*>(w_out + n * K + (int64_t)kb * kKPerBlock + 8 * wi) = *reinterpret_cast<uint4*>(out);
+  *reinterpret_cast<uint4*>(w_out + n * K + (int64_t)kb * kKPerBlock + k0) = *reinterpret_cast<uint4*>(out);
 }
 
 }  // namespace
 
-cudaError_t launch_pack(const __half* w, int64_t K, int64_t N, uint32_t* qweight, __half* scales, uint8_t* zeros,
-                        uint32_t* status, cudaStream_t stream) {
+cudaError_t launch_pack(const __half* w, int64_t K, int64_t N, int group, uint32_t* qweight, __half* scales,
+                        uint8_t* zeros, uint32_t* status, cudaStream_t stream) {
   dim3 grid((unsigned)(N / kRowsPerBlock), (unsigned)(K / kKPerBlock));
-  pack_kernel<<<grid, 512, 0, stream>>>(w, K, N, qweight, scales, zeros, status);
+  pack_kernel<<<grid, 512, 0, stream>>>(w, K, N, group, qweight, scales, zeros, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequant(const uint32_t* qweight, const __half* scales, const uint8_t* zeros, int64_t K,
-                           int64_t N, __half* w_out, cudaStream_t stream) {
+                           int64_t N, int group, __half* w_out, cudaStream_t stream) {
   dim3 grid((unsigned)(N / kRowsPerBlock), (unsigned)(K / kKPerBlock));
-  dequant_kernel<<<grid, 256, 0, stream>>>(qweight, scales, zeros, K, N, w_out);
+  dequant_kernel<<<grid, 256, 0, stream>>>(qweight, scales, zeros, K, N, group, w_out);
   return cudaGetLastError();
 }
 
