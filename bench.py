@@ -379,6 +379,65 @@ def run_ours(args):
         prefill = {"workload": f"{PREFILL[1]} K={PL.K} N={PL.N} M={Mp}", "ms": pms, "tflops_per_gpu": tflops,
                    "peak_tflops": tc_burst, "frac": tflops / tc_burst, "peak_kind": f"{peak_kind} bf16 burst"}
 
+    # ---- comparator: the same layers as dense fp16 weights through cuBLAS ----
+    # (torch.nn.functional.linear; a library call, timed the same way: CUDA
+    # graphs over rotating weight copies larger than L2). It gives the INT4 vs
+    # FP16 speedup the TinyChat README reports per token.
+    fp16 = None
+    if not args.no_fp16:
+        import torch.nn.functional as F
+        rot16 = 2
+        w16 = [[torch.from_numpy(awq_synth.layer_weight(0, wl, L).view(np.uint16)).view(torch.float16).to(dev)
+                for L in layers] for _ in range(rot16)]
+
+        def step16(r):
+            for L, x, y, w in zip(layers, xs, ys, w16[r]):
+                torch.matmul(x, w.t(), out=y)
+
+        with torch.cuda.stream(stream):
+            for r in range(rot16):
+                step16(r)
+        torch.cuda.synchronize()
+        g16 = []
+        for r in range(rot16):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step16(r)
+            g16.append(g)
+        steps16 = max(3, min(args.steps, 2000))
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                g16[i % rot16].replay()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            f0.record(stream)
+            for i in range(steps16):
+                g16[i % rot16].replay()
+            f1.record(stream)
+        barrier()
+        ms16 = max_over_ranks(f0.elapsed_time(f1)) / steps16
+        fp16 = {"library": "cuBLAS through torch.matmul, dense fp16 weights", "decode_ms_per_step": ms16,
+                "decode_speedup_int4_vs_fp16": ms16 / (ms / args.steps)}
+        del g16
+        del w16
+        if prefill is not None:
+            W = torch.from_numpy(awq_synth.layer_weight(0, pwl, PL).view(np.uint16)).view(torch.float16).to(dev)
+            for _ in range(3):
+                F.linear(xp, W, out=yp)
+            torch.cuda.synchronize()
+            q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            q0.record()
+            for _ in range(20):
+                F.linear(xp, W, out=yp)
+            q1.record()
+            torch.cuda.synchronize()
+            pms16 = max_over_ranks(q0.elapsed_time(q1)) / 20
+            fp16.update({"prefill_ms": pms16, "prefill_tflops": 2.0 * Mp * PL.N * PL.K / (pms16 * 1e-3) / 1e12,
+                         "prefill_speedup_int4_vs_fp16": pms16 / prefill["ms"]})
+            del W
+        torch.cuda.empty_cache()
+
     # ---- CPU oracle baseline on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -408,6 +467,7 @@ def run_ours(args):
         "clocks": clocks,
         "cpu_baseline": cpu,
         "prefill_gemm": prefill,
+        "fp16_comparator": fp16,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -466,6 +526,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-fp16", action="store_true", help="skip the cuBLAS fp16 comparator")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-frac", type=float, default=1.0, help="share of rows in the CPU-baseline sample")
     ap.add_argument("--ref-budget", type=float, default=60.0, help="seconds of oracle work in the reference arm")
