@@ -242,3 +242,67 @@ def test_prefill_full_size(layer, M):
     order = np.argsort(ns, kind="stable")
     y_ref, b = oracle.linear_entries(x, *hp, L.N, L.K, ms[order], ns[order])
     check_close(y[ms[order], ns[order]], y_ref, b, f"prefill/{layer} M={M}")
+
+
+# ---- decode at M <= 2, groups of 128: x as a block fixed-point integer -----
+# Each 128-input block of x is scaled by a power of two fixed by its largest
+# value and rounded to an integer below 2^30; these cases stress that step.
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_decode_one_hot_gives_the_dequantized_weight_exactly(M):
+    K, N = 1024, 336
+    W, dev, hp = _packed(N, K, "onehot12")
+    q, z, s = oracle.unpack(*hp, N, K)
+    wh = oracle.dequant(q, z, s)
+    for ks in ([0, 1], [127, 128], [300, 1023], [64, 65]):
+        x = np.zeros((M, K), np.float16)
+        for m in range(M):
+            x[m, ks[m]] = 1.0
+        y = _run(awq.awq_w4a16_gemv, x, dev, N)
+        for m in range(M):
+            assert (y[m].view(np.uint16) == wh[:, ks[m]].view(np.uint16)).all(), (M, ks[m])
+
+
+def _edge_x(kind, M, K, rng):
+    x = rng.standard_normal((M, K))
+    if kind == "outlier":      # one value per block 2^16 times the rest
+        x *= 1e-3
+        x[:, ::128] = 65.0 * np.sign(rng.standard_normal((M, K // 128)))
+    elif kind == "subnormal":  # only fp16 subnormals
+        x = rng.integers(-1023, 1024, (M, K)) * 2.0 ** -24
+    elif kind == "mixed_zero":  # whole zero blocks between normal ones
+        x[:, 128:384] = 0.0
+    elif kind == "wide":       # magnitudes from 2^-14 to 2^4 in every block (y stays finite)
+        x = np.sign(x) * 2.0 ** rng.uniform(-14, 4, (M, K))
+    return x.astype(np.float16)
+
+
+@pytest.mark.parametrize("kind", ["outlier", "subnormal", "mixed_zero", "wide"])
+@pytest.mark.parametrize("M", [1, 2])
+def test_decode_block_fixed_point_edge_cases(kind, M):
+    K, N = 2048, 592
+    W, dev, hp = _packed(N, K, "edge")
+    x = _edge_x(kind, M, K, np.random.default_rng(M))
+    y = _run(awq.awq_w4a16_gemv, x, dev, N)
+    y_ref, b = oracle.linear(x, *hp, N, K)
+    check_close(y, y_ref, b, f"{kind} M={M}")
+
+
+def test_decode_zero_activations_give_zero():
+    K, N = 2048, 592
+    W, dev, hp = _packed(N, K, "edge")
+    for M in (1, 2, 5):
+        y = _run(awq.awq_w4a16_gemv, np.zeros((M, K), np.float16), dev, N)
+        assert (y.view(np.uint16) & 0x7FFF == 0).all()
+
+
+@pytest.mark.parametrize("M", [1, 2, 5])
+@pytest.mark.parametrize("bad", [np.inf, np.nan])
+def test_decode_non_finite_activation_gives_non_finite_outputs(M, bad):
+    K, N = 1024, 336
+    W, dev, hp = _packed(N, K, "nonfin")
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, "nonfin/x"), M, K, 1.0)
+    x[M - 1, 200] = bad
+    y = _run(awq.awq_w4a16_gemv, x, dev, N).astype(np.float64)
+    assert not np.isfinite(y[M - 1]).any()
+    assert np.isfinite(y[:M - 1]).all()

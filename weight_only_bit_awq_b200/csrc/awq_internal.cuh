@@ -60,6 +60,7 @@ const DeviceInfo& device_info();   // current device
 struct GemvPlan {
   int group;            // quantization group size (128, 64 or 32)
   int nt;               // token tiles of 8 (1, 2 or 4)
+  bool int_path;        // M <= 2, groups of 128: integer MMAs on the codes and x digits
   int ku;               // k-blocks per streamed unit (1, 2 or 4)
   int stages;           // depth of the shared-memory ring
   size_t smem_bytes;    // dynamic shared memory per CTA

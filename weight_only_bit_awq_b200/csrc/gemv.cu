@@ -63,18 +63,26 @@ constexpr int kXRowBytes = kKPerBlock * 2;                        // 256 bytes o
 constexpr int kSmemPerCta2 = 112 * 1024;
 constexpr int kSmemPerCta1 = 226 * 1024;
 
+// Integer path (M <= 2, groups of 128): per k-block, the x-prep warp writes
+// the B fragments of the integer MMAs -- for each lane column t (0..3), 4 M
+// digit columns of 32 bytes, plus one 32-byte pad per t so that its stores are
+// bank-conflict free -- and one float4 of coefficients per t.
+__host__ __device__ constexpr int int_bfrag_tstride(int M) { return (4 * M + 1) * 32; }
+__host__ __device__ constexpr int int_xs_bytes(int M) { return 4 * int_bfrag_tstride(M) + 64; }
+
 // Byte offsets inside one ring stage for a unit of up to KU k-blocks, M
 // tokens and groups of GS inputs (the same numbers on the host and in every
-// thread). Scales, zeros and x sums hold one row per group of the unit.
+// thread). Scales, zeros and x sums hold one row per group of the unit; on
+// the integer path the x-sum slot of a k-block holds its B fragments.
 struct Stage {
   int q, s, z, xs, x, bytes;
-  __host__ __device__ Stage(int KU, int M, int GS) {
+  __host__ __device__ Stage(int KU, int M, int GS, bool integer = false) {
     const int rows = KU * (kKPerBlock / GS);
     q = 0;
     s = q + KU * kKbQBytes;
     z = s + rows * kKbScaleBytes;
     xs = z + rows * kKbZeroBytes;
-    x = xs + rows * kKbXsBytes;
+    x = xs + rows * (integer ? int_xs_bytes(M) : kKbXsBytes);
     bytes = x + M * KU * kXRowBytes;  // every term is a multiple of 16
   }
 };
@@ -104,6 +112,25 @@ __device__ __forceinline__ void mma_16816_first(float (&d)[4], uint32_t a0, uint
       "{%10,%10,%10,%10};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// d += A B (m16n8k32, A unsigned bytes, B signed bytes, exact s32 accumulate);
+// the _first form starts from zero.
+__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void imma_16832_first(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
 // Group size GS (128, 64 or 32) in the k-block of 128: the packed layout puts
@@ -219,6 +246,25 @@ __device__ __forceinline__ void block_mma_lohi(float (&acc)[LoHi<GS>::kAcc][4], 
   }
 }
 
+// M <= 2, groups of 128 ("integer path"): exact integer MMAs on the codes.
+// Per k-block and token, the x-prep warp writes x as a block fixed-point
+// integer, X = rint(x * 2^(44 - eb)) with eb the largest fp16 exponent field
+// of the k-block (at least 1), so |X| < 2^30 and X is exact unless |x| is
+// below 2^-19 of the k-block's largest value. X is split into four signed
+// base-256 digits, X = sum_d 256^d D_d (the bytes of (X + 0x80808080) ^
+// 0x80808080), and digit d of token m becomes column 4 m + d of the B operand
+// of mma.sync m16n8k32 (u8 x s8 -> s32): the columns an M = 1 GEMV leaves
+// idle. The codes enter operand A as bytes without conversion: word &
+// 0x0F0F0F0F gives q of inputs {0, 4, 1, 5} of the word ("lo"), word &
+// 0xF0F0F0F0 gives 16 q of {2, 6, 3, 7} ("hi"); lo and hi go to separate
+// accumulators, and the B bytes are laid out in the same k order. Per column
+// the k-block's exact integer sum is then 16 acc_lo + acc_hi = 16 sum_k q D_d,
+// so
+//   sum_k x (q - z) = sum_d 2^(eb - 48 + 8 d) (16 acc_lo + acc_hi) - z sum_k x,
+// with sum_k x in fp32 from the x-prep warp. 4 integer MMAs and 16 lop3 per
+// 2048 weights; the digit columns are added across lanes once, at the end.
+// A non-finite x sets the k-block's coefficients to NaN, so y is NaN.
+//
 // Unit numbering: UPG = ceil(KB / KU) units per group; unit u is group
 // u / UPG, k-blocks KU (u % UPG) .. min(KB, KU (u % UPG + 1)) - 1. CTA c of P
 // streams units [c U / P, (c + 1) U / P).
@@ -236,16 +282,19 @@ struct Range {
 };
 
 // kM1: M == 1 (NT == 1), where only the epilogue slots of token 0 are
-// computed. GS: group size (128, 64 or 32).
-template <int NT, int KU, bool kM1, int GS>
+// computed. GS: group size (128, 64 or 32). kInt: the integer path (NT == 1,
+// M <= 2, GS == 128).
+template <int NT, int KU, bool kM1, int GS, bool kInt>
 __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
     gemv_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight, const __half* __restrict__ scales,
                 const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M, int K, int N, int NS,
                 float* __restrict__ partial, uint32_t* status) {
   extern __shared__ __align__(16) uint8_t smem[];
-  constexpr bool kLoHi = NT == 1;
+  static_assert(!kInt || (NT == 1 && GS == 128 && !kM1), "integer path: one token tile, groups of 128");
+  constexpr bool kLoHi = NT == 1 && !kInt;
+  constexpr bool kXWarp = kLoHi || kInt;  // a ninth warp reads x first and prepares it
   constexpr int kGPK = Grp<GS>::kPerKb;  // groups per k-block
-  const Stage L(KU, M, GS);
+  const Stage L(KU, M, GS, kInt);
   const uint32_t sbase = ptx::smem_u32(smem);
   const uint32_t bar0 = sbase + NS * L.bytes;
   auto full = [&](int s) -> uint32_t { return bar0 + 8 * s; };
@@ -262,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       // 32 cp.async arrivals + 1 arrival carrying the byte count (+ 1 from the x-sum warp)
-      ptx::mbar_init(full(s), kLoHi ? 34 : 33);
+      ptx::mbar_init(full(s), kXWarp ? 34 : 33);
       ptx::mbar_init(empty(s), kConsumers);
       ptx::mbar_init(xland(s), 1);
     }
@@ -284,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
       const uint32_t st = sbase + s * L.bytes;
       if (lane == 0)
-        ptx::mbar_arrive_expect_tx(full(s), (uint32_t)(ku * R * 1024 + (kLoHi ? 0 : M * ku * kXRowBytes)));
+        ptx::mbar_arrive_expect_tx(full(s), (uint32_t)(ku * R * 1024 + (kXWarp ? 0 : M * ku * kXRowBytes)));
       __syncwarp();
       if (lane == 0)
         ptx::bulk_g2s(st + L.q, qweight + unit_first_block(cgi, kb0, rg.KB, rg.NB) * kWordsPerBlock,
@@ -308,9 +357,9 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
     auto issue_x = [&](int s) {  // activations of the next unit into stage s
       const int64_t kb0 = (int64_t)xj * KU;
       const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
-      // with the lo/hi split x lands on its own barrier: the x-sum warp reads it first
-      const uint32_t xb = kLoHi ? xland(s) : full(s);
-      if (kLoHi) {
+      // with an x-prep warp x lands on its own barrier: that warp reads it first
+      const uint32_t xb = kXWarp ? xland(s) : full(s);
+      if (kXWarp) {
         if (lane == 0) ptx::mbar_arrive_expect_tx(xb, (uint32_t)(M * ku * kXRowBytes));
         __syncwarp();
       }
@@ -391,6 +440,70 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
         }
       }
     }
+    if constexpr (kInt) {
+      // Integer path: lane (ch, hh) = (lane / 2, lane % 2) takes the 8-input
+      // chunk ch of the k-block (inputs 8 ch .. 8 ch + 7, i.e. lane column
+      // t = ch / 4, word 4 t + ch % 4 of every row) and, of it, the four
+      // inputs {0, 4, 1, 5} (hh = 0, the lo bytes of the codes) or {2, 6, 3, 7}
+      // (hh = 1, the hi bytes), in that order.
+      const int ch = lane >> 1, hh = lane & 1, tq = ch >> 2, cq = ch & 3;
+      const int tw = int_bfrag_tstride(M) / 4;       // words per lane column t
+      int jj = (int)(u0 % rg.UPG), s = 0, ph = 0;
+      for (int i = 0; i < n_units; ++i) {
+        if (!ptx::wait_bar(xland(s), ph, abort_flag, status)) break;
+        const int64_t kb0 = (int64_t)jj * KU;
+        const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
+        const uint8_t* st = smem + s * L.bytes;
+        for (int j = 0; j < ku; ++j) {
+          uint8_t* xs = smem + s * L.bytes + L.xs + j * int_xs_bytes(M);
+          uint32_t* bf = reinterpret_cast<uint32_t*>(xs) + tq * tw + hh * 4 + cq;
+          float4* coef = reinterpret_cast<float4*>(xs + 4 * int_bfrag_tstride(M));
+          for (int m = 0; m < M; ++m) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(st + L.x + (m * KU + j) * kXRowBytes + 16 * ch);
+            const uint32_t pa = hh ? xv.y : xv.x, pb = hh ? xv.w : xv.z;  // inputs (0|2, 1|3), (4|6, 5|7)
+            // largest fp16 magnitude of the k-block (bit patterns order like the values)
+            const uint32_t ma = pa & 0x7FFF7FFFu, mb = pb & 0x7FFF7FFFu;
+            const uint32_t mloc = max(max(ma & 0xFFFFu, ma >> 16), max(mb & 0xFFFFu, mb >> 16));
+            const uint32_t amax = __reduce_max_sync(0xffffffffu, mloc);
+            const int eb = max((int)(amax >> 10), 1);
+            const float sc = __int_as_float((171 - eb) << 23);  // 2^(44 - eb), exact scaling
+            const float2 fa = __half22float2(u32_as_h2(pa)), fb = __half22float2(u32_as_h2(pb));
+            // X in the k order {0, 4, 1, 5} / {2, 6, 3, 7}; digits as the bytes of v
+            const uint32_t v0 = ((uint32_t)__float2int_rn(fa.x * sc) + 0x80808080u) ^ 0x80808080u;
+            const uint32_t v1 = ((uint32_t)__float2int_rn(fb.x * sc) + 0x80808080u) ^ 0x80808080u;
+            const uint32_t v2 = ((uint32_t)__float2int_rn(fa.y * sc) + 0x80808080u) ^ 0x80808080u;
+            const uint32_t v3 = ((uint32_t)__float2int_rn(fb.y * sc) + 0x80808080u) ^ 0x80808080u;
+            // 4 x 4 byte transpose: D_d = digit d of the four inputs
+            const uint32_t t01l = __byte_perm(v0, v1, 0x5140), t01h = __byte_perm(v0, v1, 0x7362);
+            const uint32_t t23l = __byte_perm(v2, v3, 0x5140), t23h = __byte_perm(v2, v3, 0x7362);
+            uint32_t* b = bf + 4 * m * 8;  // column 4 m + d at + 8 d words
+            b[0] = __byte_perm(t01l, t23l, 0x5410);
+            b[8] = __byte_perm(t01l, t23l, 0x7632);
+            b[16] = __byte_perm(t01h, t23h, 0x5410);
+            b[24] = __byte_perm(t01h, t23h, 0x7632);
+            float cs = (fa.x + fa.y) + (fb.x + fb.y);
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
+            // lane column t' = 2 m + e holds digit columns 4 m + 2 e, 4 m + 2 e + 1:
+            // {2^(eb - 48 + 8 d0), sum x if d0 == 0, 2^(eb - 48 + 8 d0 + 8), 0}
+            if (lane >> 1 == m) {
+              const int d0 = 2 * (lane & 1);
+              float f0 = __int_as_float((eb + 79 + 8 * d0) << 23), f1 = __int_as_float((eb + 87 + 8 * d0) << 23);
+              if (amax >= 0x7C00u) f0 = f1 = __int_as_float(0x7FC00000);  // inf or NaN in x: y is NaN
+              coef[lane] = make_float4(f0, d0 == 0 ? cs : 0.f, f1, 0.f);
+            }
+          }
+          if (M == 1 && (lane == 2 || lane == 3)) coef[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(full(s));
+        if (++jj == rg.UPG) jj = 0;
+        if (++s == NS) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
     return;
   }
 
@@ -431,10 +544,63 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
   // else this CTA's fp32 partial sums, which the fixup kernel adds up.
   auto finish_group = [&](int64_t g_, const float (&v)[NT][4]) {
     if (cw >= group_rows(g_, rg.NB)) return;
+    if constexpr (kInt) {
+      // add the digit columns: lane t holds columns 2t, 2t+1 (token t / 2),
+      // so after the pair sum lanes t = 0 and t = 2 hold tokens 0 and 1
+      float r0 = v[0][0] + v[0][1], r1 = v[0][2] + v[0][3];
+      r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+      const int m = t >> 1;
+      if ((t & 1) || m >= M) return;
+      const int64_t ra = (g_ * kGroupBlocks + cw) * kRowsPerBlock + g;
+      if (covered(g_)) {
+        y[(int64_t)m * N + ra] = __float2half_rn(r0);
+        y[(int64_t)m * N + ra + 8] = __float2half_rn(r1);
+      } else {
+        float* mine = slot(c, g_);
+        mine[g * M + m] = r0;
+        mine[(g + 8) * M + m] = r1;
+      }
+      return;
+    }
     if (covered(g_))
       write_y(g_, v);
     else
       store_partial(g_, v);
+  };
+
+  // ---- integer path: one k-block (index j of the unit in stage st) ----
+  auto kblock_int = [&](const uint8_t* st, int j, int R) {
+    const uint8_t* blk = st + L.q + (j * R + cw) * 1024;
+    const uint4 wa = *reinterpret_cast<const uint4*>(blk + g * 64 + 16 * t);
+    const uint4 wb = *reinterpret_cast<const uint4*>(blk + (g + 8) * 64 + 16 * t);
+    const uint8_t* xs = st + L.xs + j * int_xs_bytes(M);
+    // B fragments of lane (g, t): digit column g, lane column t; zero past the tokens
+    uint4 xb0 = make_uint4(0, 0, 0, 0), xb1 = make_uint4(0, 0, 0, 0);
+    if (g < 4 * M) {
+      const uint8_t* bf = xs + t * int_bfrag_tstride(M) + g * 32;
+      xb0 = *reinterpret_cast<const uint4*>(bf);
+      xb1 = *reinterpret_cast<const uint4*>(bf + 16);
+    }
+    const float4 cf = *reinterpret_cast<const float4*>(xs + 4 * int_bfrag_tstride(M) + 16 * t);
+    const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + L.s + j * kKbScaleBytes) + cw * kRowsPerBlock;
+    const uint8_t* zr = st + L.z + j * kKbZeroBytes + cw * (kRowsPerBlock / 2);
+    const float sr[2] = {pos_half_bits_to_float(sc[g]), pos_half_bits_to_float(sc[g + 8])};
+    const uint32_t za = (zr[g >> 1] >> (4 * (g & 1))) & 0xF, zb = (zr[(g + 8) >> 1] >> (4 * (g & 1))) & 0xF;
+    const float zf[2] = {__uint_as_float(0x4B000000u | za) - 8388608.f,  // exact (float)z
+                         __uint_as_float(0x4B000000u | zb) - 8388608.f};
+    constexpr uint32_t kLo = 0x0F0F0F0Fu, kHi = 0xF0F0F0F0u;
+    int acc_lo[4], acc_hi[4];
+    imma_16832_first(acc_lo, wa.x & kLo, wb.x & kLo, wa.y & kLo, wb.y & kLo, xb0.x, xb0.y);
+    imma_16832_first(acc_hi, wa.x & kHi, wb.x & kHi, wa.y & kHi, wb.y & kHi, xb1.x, xb1.y);
+    imma_16832(acc_lo, wa.z & kLo, wb.z & kLo, wa.w & kLo, wb.w & kLo, xb0.z, xb0.w);
+    imma_16832(acc_hi, wa.z & kHi, wb.z & kHi, wa.w & kHi, wb.w & kHi, xb1.z, xb1.w);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const float f = (cc & 1) ? cf.z : cf.x, cx = (cc & 1) ? cf.w : cf.y;
+      const float v = __int2float_rn(acc_lo[cc] * 16 + acc_hi[cc]);  // exact: |.| < 2^22
+      yacc[0][cc] = fmaf(sr[cc >> 1], fmaf(f, v, -zf[cc >> 1] * cx), yacc[0][cc]);
+    }
   };
 
   // ---- one k-block (index j of the unit in stage st) of this warp's row block ----
@@ -524,10 +690,14 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
   };
 
   auto kblock = [&](const uint8_t* st, int j, int R) {
-    Acc acc;
-    KState ks;
-    kb_issue(st, j, R, acc, ks);
-    kb_finish(acc, ks);
+    if constexpr (kInt) {
+      kblock_int(st, j, R);
+    } else {
+      Acc acc;
+      KState ks;
+      kb_issue(st, j, R, acc, ks);
+      kb_finish(acc, ks);
+    }
   };
 
   bool ok = true;
@@ -610,14 +780,14 @@ __global__ void __launch_bounds__(128) gemv_fixup_kernel(const float* __restrict
   y[(int64_t)m * N + gi * kGroupBlocks * kRowsPerBlock + threadIdx.x] = __float2half_rn(v);
 }
 
-template <int NT, int KU, bool kM1, int GS>
+template <int NT, int KU, bool kM1, int GS, bool kInt>
 cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros, __half* y,
                      int M, int K, int N, void* workspace, const GemvPlan& p, cudaStream_t stream) {
   static uint64_t attr_set = 0;  // one bit per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
   if (!(attr_set >> dev & 1)) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, KU, kM1, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, KU, kM1, GS, kInt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          NT == 4 ? kSmemPerCta1 : kSmemPerCta2);
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
@@ -635,7 +805,7 @@ cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* sca
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<NT, KU, kM1, GS>, x, qweight, scales, zeros, y, M, K, N, p.stages,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<NT, KU, kM1, GS, kInt>, x, qweight, scales, zeros, y, M, K, N, p.stages,
                                      partial, status);
   if (e != cudaSuccess || !p.has_split) return e;
   cudaLaunchConfig_t fcfg = cfg;
@@ -645,13 +815,13 @@ cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* sca
   return cudaLaunchKernelEx(&fcfg, gemv_fixup_kernel, (const float*)partial, y, M, K, N, p.ku, p.ctas);
 }
 
-template <int NT, bool kM1, int GS>
+template <int NT, bool kM1, int GS, bool kInt = false>
 cudaError_t launch_nt(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
                       __half* y, int M, int K, int N, void* workspace, const GemvPlan& p, cudaStream_t stream) {
   switch (p.ku) {
-    case 1: return launch_t<NT, 1, kM1, GS>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
-    case 2: return launch_t<NT, 2, kM1, GS>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
-    case 4: return launch_t<NT, 4, kM1, GS>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    case 1: return launch_t<NT, 1, kM1, GS, kInt>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    case 2: return launch_t<NT, 2, kM1, GS, kInt>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
+    case 4: return launch_t<NT, 4, kM1, GS, kInt>(x, qweight, scales, zeros, y, M, K, N, workspace, p, stream);
     default: return cudaErrorInvalidConfiguration;
   }
 }
@@ -659,6 +829,9 @@ cudaError_t launch_nt(const __half* x, const uint32_t* qweight, const __half* sc
 template <int GS>
 cudaError_t launch_g(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
                      __half* y, int m, int k, int n, void* workspace, const GemvPlan& p, cudaStream_t stream) {
+  if constexpr (GS == 128) {
+    if (p.int_path) return launch_nt<1, false, GS, true>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream);
+  }
   switch (p.nt) {
     case 1:
       return m == 1 ? launch_nt<1, true, GS>(x, qweight, scales, zeros, y, m, k, n, workspace, p, stream)
@@ -682,6 +855,7 @@ GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int group, int sm_count) {
   GemvPlan p{};
   p.group = group;
   p.nt = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
+  p.int_path = M <= 2 && group == 128;
   const int64_t NB = N / kRowsPerBlock, KB = K / kKPerBlock;
   p.groups = (int)((NB + kGroupBlocks - 1) / kGroupBlocks);
   const int64_t per_sm = p.nt == 4 ? 1 : 2;  // resident CTAs per SM (shared memory and registers)
@@ -689,7 +863,7 @@ GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int group, int sm_count) {
   const int64_t Mi = M < 1 ? 1 : M;
   for (int ku : {4, 2, 1}) {
     const int64_t U = p.groups * ((KB + ku - 1) / ku);
-    const int stage = Stage(ku, (int)Mi, group).bytes;
+    const int stage = Stage(ku, (int)Mi, group, p.int_path).bytes;
     int stages = budget / stage;
     if (stages > kMaxStages) stages = kMaxStages;
     const bool last = ku == 1;
