@@ -129,8 +129,13 @@ awq_status awq_dequant(const void* qweight, const void* scales, const void* zero
 
 /* Decode-stage W4A16 GEMV, 1 <= M <= AWQ_GEMV_MAX_M (README "Speed
  * Benchmarks": per-token latency of the generation stage): y fp16 [M][N] =
- * x fp16 [M][K] . W^T. Streams the packed weights once; fp32 accumulation.
- * M > AWQ_GEMV_MAX_M returns AWQ_ERR_UNSUPPORTED. */
+ * x fp16 [M][K] . W^T. Streams the packed weights once; fp32 accumulation
+ * (M <= 2 with groups of 128: exact integer sums of the codes times a block
+ * fixed-point form of x, exact except for inputs below 2^-19 of their
+ * 128-input block's largest magnitude). Rows whose k-range is split between
+ * CTAs are added in a fixed order, so results are deterministic. A non-finite
+ * x[m][k] gives non-finite y[m][*]. M > AWQ_GEMV_MAX_M returns
+ * AWQ_ERR_UNSUPPORTED. */
 awq_status awq_w4a16_gemv(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
                           int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,
                           void* stream);

@@ -451,23 +451,26 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       int jj = (int)(u0 % rg.UPG), s = 0, ph = 0;
       for (int i = 0; i < n_units; ++i) {
         if (!ptx::wait_bar(xland(s), ph, abort_flag, status)) break;
-        const int64_t kb0 = (int64_t)jj * KU;
-        const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
         const uint8_t* st = smem + s * L.bytes;
-        for (int j = 0; j < ku; ++j) {
-          uint8_t* xs = smem + s * L.bytes + L.xs + j * int_xs_bytes(M);
-          uint32_t* bf = reinterpret_cast<uint32_t*>(xs) + tq * tw + hh * 4 + cq;
-          float4* coef = reinterpret_cast<float4*>(xs + 4 * int_bfrag_tstride(M));
-          for (int m = 0; m < M; ++m) {
+        // All KU k-blocks of the stage at once (their latency chains overlap);
+        // slots past a short last unit get values that are never read.
+        for (int m = 0; m < M; ++m) {
+          uint32_t pa[KU], pb[KU], amax[KU];
+#pragma unroll
+          for (int j = 0; j < KU; ++j) {
             const uint4 xv = *reinterpret_cast<const uint4*>(st + L.x + (m * KU + j) * kXRowBytes + 16 * ch);
-            const uint32_t pa = hh ? xv.y : xv.x, pb = hh ? xv.w : xv.z;  // inputs (0|2, 1|3), (4|6, 5|7)
+            pa[j] = hh ? xv.y : xv.x;  // inputs (0|2, 1|3)
+            pb[j] = hh ? xv.w : xv.z;  // inputs (4|6, 5|7)
             // largest fp16 magnitude of the k-block (bit patterns order like the values)
-            const uint32_t ma = pa & 0x7FFF7FFFu, mb = pb & 0x7FFF7FFFu;
-            const uint32_t mloc = max(max(ma & 0xFFFFu, ma >> 16), max(mb & 0xFFFFu, mb >> 16));
-            const uint32_t amax = __reduce_max_sync(0xffffffffu, mloc);
-            const int eb = max((int)(amax >> 10), 1);
+            const uint32_t ma = pa[j] & 0x7FFF7FFFu, mb = pb[j] & 0x7FFF7FFFu;
+            amax[j] = __reduce_max_sync(0xffffffffu, max(max(ma & 0xFFFFu, ma >> 16), max(mb & 0xFFFFu, mb >> 16)));
+          }
+          float cs[KU];
+#pragma unroll
+          for (int j = 0; j < KU; ++j) {
+            const int eb = max((int)(amax[j] >> 10), 1);
             const float sc = __int_as_float((171 - eb) << 23);  // 2^(44 - eb), exact scaling
-            const float2 fa = __half22float2(u32_as_h2(pa)), fb = __half22float2(u32_as_h2(pb));
+            const float2 fa = __half22float2(u32_as_h2(pa[j])), fb = __half22float2(u32_as_h2(pb[j]));
             // X in the k order {0, 4, 1, 5} / {2, 6, 3, 7}; digits as the bytes of v
             const uint32_t v0 = ((uint32_t)__float2int_rn(fa.x * sc) + 0x80808080u) ^ 0x80808080u;
             const uint32_t v1 = ((uint32_t)__float2int_rn(fb.x * sc) + 0x80808080u) ^ 0x80808080u;
@@ -476,24 +479,38 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
             // 4 x 4 byte transpose: D_d = digit d of the four inputs
             const uint32_t t01l = __byte_perm(v0, v1, 0x5140), t01h = __byte_perm(v0, v1, 0x7362);
             const uint32_t t23l = __byte_perm(v2, v3, 0x5140), t23h = __byte_perm(v2, v3, 0x7362);
-            uint32_t* b = bf + 4 * m * 8;  // column 4 m + d at + 8 d words
+            uint32_t* b = reinterpret_cast<uint32_t*>(smem + s * L.bytes + L.xs + j * int_xs_bytes(M)) + tq * tw +
+                          hh * 4 + cq + 4 * m * 8;  // column 4 m + d at + 8 d words
             b[0] = __byte_perm(t01l, t23l, 0x5410);
             b[8] = __byte_perm(t01l, t23l, 0x7632);
             b[16] = __byte_perm(t01h, t23h, 0x5410);
             b[24] = __byte_perm(t01h, t23h, 0x7632);
-            float cs = (fa.x + fa.y) + (fb.x + fb.y);
+            cs[j] = (fa.x + fa.y) + (fb.x + fb.y);
+          }
 #pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
-            // lane column t' = 2 m + e holds digit columns 4 m + 2 e, 4 m + 2 e + 1:
-            // {2^(eb - 48 + 8 d0), sum x if d0 == 0, 2^(eb - 48 + 8 d0 + 8), 0}
-            if (lane >> 1 == m) {
-              const int d0 = 2 * (lane & 1);
+          for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+            for (int j = 0; j < KU; ++j) cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], off);
+          // lane column t' = 2 m + e holds digit columns 4 m + 2 e, 4 m + 2 e + 1:
+          // {2^(eb - 48 + 8 d0), sum x if d0 == 0, 2^(eb - 48 + 8 d0 + 8), 0}
+          if (lane >> 1 == m) {
+            const int d0 = 2 * (lane & 1);
+#pragma unroll
+            for (int j = 0; j < KU; ++j) {
+              const int eb = max((int)(amax[j] >> 10), 1);
               float f0 = __int_as_float((eb + 79 + 8 * d0) << 23), f1 = __int_as_float((eb + 87 + 8 * d0) << 23);
-              if (amax >= 0x7C00u) f0 = f1 = __int_as_float(0x7FC00000);  // inf or NaN in x: y is NaN
-              coef[lane] = make_float4(f0, d0 == 0 ? cs : 0.f, f1, 0.f);
+              if (amax[j] >= 0x7C00u) f0 = f1 = __int_as_float(0x7FC00000);  // inf or NaN in x: y is NaN
+              float4* coef = reinterpret_cast<float4*>(smem + s * L.bytes + L.xs + j * int_xs_bytes(M) +
+                                                       4 * int_bfrag_tstride(M));
+              coef[lane] = make_float4(f0, d0 == 0 ? cs[j] : 0.f, f1, 0.f);
             }
           }
-          if (M == 1 && (lane == 2 || lane == 3)) coef[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (M == 1 && (lane == 2 || lane == 3)) {
+#pragma unroll
+          for (int j = 0; j < KU; ++j)
+            reinterpret_cast<float4*>(smem + s * L.bytes + L.xs + j * int_xs_bytes(M) + 4 * int_bfrag_tstride(M))[lane] =
+                make_float4(0.f, 0.f, 0.f, 0.f);
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(full(s));
@@ -526,8 +543,9 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       }
   };
   // Partial slot of CTA `cta` for group g_: [cta][first/last group of cta][row block][16 rows][M].
+  const int64_t first_gi = u0 / rg.UPG;  // this CTA's first group
   auto slot = [&](int64_t cta, int64_t g_) -> float* {
-    const int which = (g_ == rg.first_unit(cta) / rg.UPG) ? 0 : 1;
+    const int which = (g_ == first_gi) ? 0 : 1;
     return partial + ((cta * 2 + which) * kGroupBlocks + cw) * kRowsPerBlock * M;
   };
   auto store_partial = [&](int64_t g_, const float (&v)[NT][4]) {
@@ -750,7 +768,9 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
 // row), launched right after the GEMV in the same stream. It waits for the
 // GEMV's writes (programmatic dependent launch), adds the contributors'
 // partial slots in CTA order and writes fp16 y. Groups that one CTA covered
-// exit.
+// exit. Every contributor but the first starts its range inside the group, so
+// the group is its first one (slot 0); the first contributor holds the group
+// in slot 0 only if its range starts exactly at the group's first unit.
 __global__ void __launch_bounds__(128) gemv_fixup_kernel(const float* __restrict__ partial, __half* __restrict__ y,
                                                           int M, int K, int N, int KU, int P) {
   ptx::griddep_launch_dependents();
@@ -761,19 +781,17 @@ __global__ void __launch_bounds__(128) gemv_fixup_kernel(const float* __restrict
   const int rb = threadIdx.x >> 4, row = threadIdx.x & 15;
   if (rb >= group_rows(gi, rg.NB)) return;
   const int m = blockIdx.y;
+  const int64_t slot_floats = (int64_t)kGroupBlocks * kRowsPerBlock * M;  // one slot
+  const int64_t cta_floats = 2 * slot_floats;                             // one CTA's two slots
+  const float* p = partial + c_first * cta_floats + ((int64_t)rb * kRowsPerBlock + row) * M + m;
+  const int which_first = rg.first_unit(c_first) == gi * rg.UPG ? 0 : 1;
+  const int n = (int)(c_last - c_first);  // contributors after the first
   ptx::griddep_wait();
-  float v = 0.f;
-  for (int64_t q0 = c_first; q0 <= c_last; q0 += 8) {
+  float v = __ldcg(p + which_first * slot_floats);
+  for (int q0 = 1; q0 <= n; q0 += 8) {
     float part[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int64_t q = q0 + k;
-      part[k] = 0.f;
-      if (q <= c_last) {
-        const int which = (gi == rg.first_unit(q) / rg.UPG) ? 0 : 1;
-        part[k] = __ldcg(partial + (((q * 2 + which) * kGroupBlocks + rb) * kRowsPerBlock + row) * M + m);
-      }
-    }
+    for (int k = 0; k < 8; ++k) part[k] = q0 + k <= n ? __ldcg(p + (int64_t)(q0 + k) * cta_floats) : 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) v += part[k];
   }
@@ -805,8 +823,8 @@ cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* sca
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<NT, KU, kM1, GS, kInt>, x, qweight, scales, zeros, y, M, K, N, p.stages,
-                                     partial, status);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<NT, KU, kM1, GS, kInt>, x, qweight, scales, zeros, y, M, K, N,
+                                     p.stages, partial, status);
   if (e != cudaSuccess || !p.has_split) return e;
   cudaLaunchConfig_t fcfg = cfg;
   fcfg.gridDim = dim3((unsigned)p.groups, (unsigned)M);
