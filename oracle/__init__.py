@@ -17,7 +17,10 @@ exhaustive fp16 conversion against numpy/torch, exactly representable groups
 grid-point brute force over all 16 codes, hand-derived tie cases
 (tests/golden/), pack/unpack round trips and a hand-derived packed word, one-
 hot activations, a second factored matmul route, numpy's fp64 matmul and
-exact rational arithmetic on tiny shapes.
+exact rational arithmetic on tiny shapes. The W4A8-FP8 functions
+(tests/test_oracle_fp8.py) are pinned to torch's float8_e4m3fn decoding and
+in-range rounding, hand-derived ties, saturation and exponent cases, and a
+closed-form bound against the W4A16 layer.
 """
 from __future__ import annotations
 
@@ -73,8 +76,19 @@ def _load():
             lib.orc_linear_rows.argtypes = [vp, i64, vp, vp, vp, i64, i64, ci, i64, i64, vp, vp]
             lib.orc_linear.argtypes = [vp, i64, vp, vp, vp, i64, i64, ci, vp, vp]
             lib.orc_linear_entries.argtypes = [vp, i64, vp, vp, vp, i64, i64, ci, vp, vp, i64, vp, vp]
+            lib.orc_e4m3_to_double.restype = ctypes.c_double
+            lib.orc_e4m3_to_double.argtypes = [ctypes.c_uint8]
+            lib.orc_double_to_e4m3.restype = ctypes.c_uint8
+            lib.orc_double_to_e4m3.argtypes = [ctypes.c_double]
+            lib.orc_fp8_quantize_x.argtypes = [vp, i64, i64, vp, vp]
+            lib.orc_fp8_row_exponents.argtypes = [vp, i64, i64, ci, vp]
+            lib.orc_fp8_weights.argtypes = [vp, vp, vp, vp, i64, i64, ci, vp]
+            lib.orc_fp8_linear_rows.argtypes = [vp, vp, i64, vp, vp, vp, vp, i64, i64, ci, i64, i64, vp, vp]
+            lib.orc_fp8_linear_entries.argtypes = [vp, vp, i64, vp, vp, vp, vp, i64, i64, ci, vp, vp, i64, vp, vp]
             for f in ("orc_quantize", "orc_dequant", "orc_pack", "orc_unpack", "orc_matmul",
-                      "orc_matmul_factored", "orc_linear_rows", "orc_linear", "orc_linear_entries"):
+                      "orc_matmul_factored", "orc_linear_rows", "orc_linear", "orc_linear_entries",
+                      "orc_fp8_quantize_x", "orc_fp8_row_exponents", "orc_fp8_weights", "orc_fp8_linear_rows",
+                      "orc_fp8_linear_entries"):
                 getattr(lib, f).restype = ci
             _lib = lib
     return _lib
@@ -208,4 +222,70 @@ def linear_entries(x, qweight, scales, zeros, N: int, K: int, ms, ns, group: int
     _check(_load().orc_linear_entries(_p(xb), M, _p(np.ascontiguousarray(qweight)), _p(_bits(scales)),
                                       _p(np.ascontiguousarray(zeros)), N, K, group, _p(ms), _p(ns), len(ms),
                                       _p(y), _p(b)), "linear_entries")
+    return y, b
+
+
+# -- W4A8-FP8 variant (E4M3 activations and weights) --------------------------
+
+def e4m3_to_double(code: int) -> float:
+    return float(_load().orc_e4m3_to_double(int(code)))
+
+
+def double_to_e4m3(d: float) -> int:
+    """Nearest E4M3 value (ties to even), saturating at +-448; NaN -> 0x7F."""
+    return int(_load().orc_double_to_e4m3(float(d)))
+
+
+def fp8_quantize_x(x):
+    """x fp16 [M][K] -> (x8 uint8 E4M3 codes [M][K], sx float32 [M])."""
+    xb = _bits(x)
+    M, K = xb.shape
+    x8 = np.empty((M, K), np.uint8)
+    sx = np.empty(M, np.float32)
+    _check(_load().orc_fp8_quantize_x(_p(xb), M, K, _p(x8), _p(sx)), "fp8_quantize_x")
+    return x8, sx
+
+
+def fp8_row_exponents(scales, N: int, K: int, group: int = 128) -> np.ndarray:
+    """int8 [N]: the largest e with 15 * max_g s[n] * 2^e <= 448."""
+    e = np.empty(N, np.int8)
+    _check(_load().orc_fp8_row_exponents(_p(_bits(scales)), N, K, group, _p(e)), "fp8_row_exponents")
+    return e
+
+
+def fp8_weights(qweight, scales, zeros, e, N: int, K: int, group: int = 128) -> np.ndarray:
+    """uint8 [N][K]: E4M3 codes of W^[n,k] * 2^e[n]."""
+    w8 = np.empty((N, K), np.uint8)
+    _check(_load().orc_fp8_weights(_p(np.ascontiguousarray(qweight)), _p(_bits(scales)),
+                                   _p(np.ascontiguousarray(zeros)), _p(np.ascontiguousarray(e, dtype=np.int8)),
+                                   N, K, group, _p(w8)), "fp8_weights")
+    return w8
+
+
+def fp8_linear(x8, sx, qweight, scales, zeros, e, N: int, K: int, group: int = 128, rows: tuple | None = None):
+    """y, B (fp64) of the W4A8-FP8 layer for all rows, or rows n0..n1-1."""
+    x8 = np.ascontiguousarray(x8, dtype=np.uint8)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    M = x8.shape[0]
+    n0, n1 = (0, N) if rows is None else rows
+    y = np.empty((M, n1 - n0), np.float64)
+    b = np.empty((M, n1 - n0), np.float64)
+    _check(_load().orc_fp8_linear_rows(_p(x8), _p(sx), M, _p(np.ascontiguousarray(qweight)), _p(_bits(scales)),
+                                       _p(np.ascontiguousarray(zeros)), _p(np.ascontiguousarray(e, dtype=np.int8)),
+                                       N, K, group, n0, n1, _p(y), _p(b)), "fp8_linear")
+    return y, b
+
+
+def fp8_linear_entries(x8, sx, qweight, scales, zeros, e, N: int, K: int, ms, ns, group: int = 128):
+    x8 = np.ascontiguousarray(x8, dtype=np.uint8)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    M = x8.shape[0]
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    y = np.empty(len(ms), np.float64)
+    b = np.empty(len(ms), np.float64)
+    _check(_load().orc_fp8_linear_entries(_p(x8), _p(sx), M, _p(np.ascontiguousarray(qweight)), _p(_bits(scales)),
+                                          _p(np.ascontiguousarray(zeros)),
+                                          _p(np.ascontiguousarray(e, dtype=np.int8)), N, K, group, _p(ms), _p(ns),
+                                          len(ms), _p(y), _p(b)), "fp8_linear_entries")
     return y, b

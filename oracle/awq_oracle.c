@@ -47,6 +47,9 @@
  *       scales   fp16  [K/G][N]
  *       zeros    uint8 [K/G][N/2]: low nibble = even n, high nibble = odd n.
  *
+ * A W4A8-FP8 variant (E4M3 activations and weights, fp32 accumulation) is at
+ * the end of the file, with its own statement of what it computes.
+ *
  * fp16 conversions below are written from the IEEE 754 binary16 definition
  * (1 sign bit, 5 exponent bits with bias 15, 10 fraction bits; exponent field
  * 0 encodes subnormals f * 2^-24).
@@ -340,6 +343,176 @@ int orc_linear_entries(const uint16_t* x, int64_t M, const uint32_t* qweight, co
     double acc = 0.0, b = 0.0;
     for (int64_t k = 0; k < K; ++k) {
       double p = orc_half_to_double(x[m * K + k]) * row[k];
+      acc += p;
+      b += fabs(p);
+    }
+    y[i] = acc;
+    if (bound) bound[i] = b;
+  }
+  free(row);
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* W4A8-FP8 variant                                                           */
+/* ------------------------------------------------------------------------- */
+/*
+ * The TensorRT-LLM news item on INT4 AWQ on one H200 says its AWQ kernels
+ * compute in FP8 on Hopper's tensor cores. The pages give no recipe; this is
+ * the plainest reading, with the 4-bit weights and their fp16 group scales
+ * unchanged:
+ *   - activations: per token m, sx[m] = fp32(amax_k |x[m,k]|) / 448 and
+ *     x8[m,k] = e4m3(x[m,k] / sx[m]), both divisions IEEE binary32 (448 is the
+ *     largest finite E4M3 value); a row of zeros gives sx = 0 and x8 = 0.
+ *   - weights: per output channel n, S_n = max over its groups of s, and e[n]
+ *     the largest integer with 15 * S_n * 2^e <= 448 (every |q - z| <= 15, so
+ *     W^ * 2^e stays within the E4M3 range); W8[n,k] = e4m3(W^[n,k] * 2^e[n]).
+ *   - y[m,n] = sum_k (x8[m,k] sx[m]) (W8[n,k] 2^-e[n]), here in fp64.
+ * e4m3(v) rounds v to the nearest E4M3 value, ties to even, and saturates:
+ * |v| >= 448 (or infinite) gives +-448; NaN gives 0x7F.
+ *
+ * E4M3 (OCP 8-bit floating point, the "FN" variant): 1 sign bit, 4 exponent
+ * bits with bias 7, 3 fraction bits, no infinities; exponent field 0 encodes
+ * subnormals f * 2^-9; exponent 15 with fraction 7 is NaN (0x7F, 0xFF), so
+ * the largest finite value is 1.75 * 2^8 = 448.
+ */
+
+double orc_e4m3_to_double(uint8_t b) {
+  int sign = (b >> 7) & 1;
+  int e = (b >> 3) & 0xF;
+  int f = b & 7;
+  double v;
+  if (e == 15 && f == 7)
+    v = NAN;
+  else if (e == 0)
+    v = ldexp((double)f, -9);               /* subnormal: f * 2^-9 */
+  else
+    v = ldexp((double)(8 + f), e - 10);     /* (1 + f/8) * 2^(e-7) */
+  return sign ? -v : v;
+}
+
+uint8_t orc_double_to_e4m3(double d) {
+  if (isnan(d)) return 0x7F;
+  uint8_t sign = signbit(d) ? 0x80 : 0x00;
+  double a = fabs(d);
+  if (a >= 448.0) return sign | 0x7E;       /* saturate (infinities too) */
+  if (a < ldexp(1.0, -6)) {
+    /* subnormal spacing 2^-9: n = rint(a / 2^-9) in 0..8; n = 8 is the
+       smallest normal value (code 0x08) */
+    double n = rint(ldexp(a, 9));
+    return sign | (uint8_t)n;
+  }
+  int ex;
+  frexp(a, &ex);                            /* a = m 2^ex, m in [0.5, 1) */
+  int e = ex - 1;                           /* 2^e <= a < 2^(e+1), e in -6 .. 8 */
+  double n = rint(ldexp(a, 3 - e));         /* a / 2^(e-3), in 8 .. 16 */
+  if (n == 16.0) { n = 8.0; ++e; }
+  uint8_t code = (uint8_t)(((e + 7) << 3) | ((int)n - 8));
+  if (code > 0x7E) code = 0x7E;
+  return sign | code;
+}
+
+/* x8 [M][K] E4M3 codes and sx [M] (fp32) from x fp16 [M][K]. */
+int orc_fp8_quantize_x(const uint16_t* x, int64_t M, int64_t K, uint8_t* x8, float* sx) {
+  if (M < 0 || K <= 0) return ORC_ERR_SHAPE;
+  for (int64_t m = 0; m < M; ++m) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+      float a = (float)fabs(orc_half_to_double(x[m * K + k]));   /* exact: fp16 values are fp32 values */
+      if (a > amax || isnan(a)) amax = a;
+    }
+    volatile float s = amax / 448.0f;   /* one IEEE binary32 division */
+    sx[m] = s;
+    for (int64_t k = 0; k < K; ++k) {
+      if (s == 0.0f) { x8[m * K + k] = 0; continue; }
+      volatile float v = (float)orc_half_to_double(x[m * K + k]) / s;   /* one IEEE binary32 division */
+      x8[m * K + k] = orc_double_to_e4m3((double)v);
+    }
+  }
+  return ORC_OK;
+}
+
+/* e [N] from scales fp16 [K/G][N] (packed layout). */
+int orc_fp8_row_exponents(const uint16_t* scales, int64_t N, int64_t K, int G, int8_t* e) {
+  if (bad_shape(N, K, G)) return ORC_ERR_SHAPE;
+  for (int64_t n = 0; n < N; ++n) {
+    double S = 0.0;
+    for (int64_t g = 0; g < K / G; ++g) {
+      double s = orc_half_to_double(scales[g * N + n]);
+      if (s > S) S = s;
+    }
+    int ee = 0;
+    if (S > 0.0) {
+      int ex;
+      frexp(448.0 / (15.0 * S), &ex);
+      ee = ex - 1;                                         /* close to the answer */
+      while (15.0 * ldexp(S, ee + 1) <= 448.0) ++ee;        /* exact: S 2^e is exact in fp64 */
+      while (15.0 * ldexp(S, ee) > 448.0) --ee;
+    }
+    e[n] = (int8_t)ee;
+  }
+  return ORC_OK;
+}
+
+/* W8 [N][K] E4M3 codes of the packed weight scaled by 2^e[n]. */
+int orc_fp8_weights(const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros, const int8_t* e,
+                    int64_t N, int64_t K, int G, uint8_t* w8) {
+  if (bad_shape(N, K, G) || word_in_row(0, G) < 0) return ORC_ERR_SHAPE;
+  double* row = (double*)malloc(sizeof(double) * (size_t)K);
+  for (int64_t n = 0; n < N; ++n) {
+    packed_row(qweight, scales, zeros, N, K, G, n, row);
+    for (int64_t k = 0; k < K; ++k) w8[n * K + k] = orc_double_to_e4m3(ldexp(row[k], e[n]));
+  }
+  free(row);
+  return ORC_OK;
+}
+
+/* Row n of the W4A8-FP8 weight as the values it stands for: W8[n,k] 2^-e[n]. */
+static void fp8_row(const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros, const int8_t* e,
+                    int64_t N, int64_t K, int G, int64_t n, double* row) {
+  packed_row(qweight, scales, zeros, N, K, G, n, row);
+  for (int64_t k = 0; k < K; ++k) row[k] = ldexp(orc_e4m3_to_double(orc_double_to_e4m3(ldexp(row[k], e[n]))), -e[n]);
+}
+
+/* y, bound [M][n1-n0]: output channels n0..n1-1 of the W4A8-FP8 layer, from
+ * x8, sx and the packed buffers, in fp64 in increasing k. */
+int orc_fp8_linear_rows(const uint8_t* x8, const float* sx, int64_t M, const uint32_t* qweight,
+                        const uint16_t* scales, const uint8_t* zeros, const int8_t* e, int64_t N, int64_t K, int G,
+                        int64_t n0, int64_t n1, double* y, double* bound) {
+  if (M < 0 || bad_shape(N, K, G) || word_in_row(0, G) < 0 || n0 < 0 || n1 > N || n0 > n1) return ORC_ERR_SHAPE;
+  int64_t W = n1 - n0;
+  double* row = (double*)malloc(sizeof(double) * (size_t)K);
+  for (int64_t n = n0; n < n1; ++n) {
+    fp8_row(qweight, scales, zeros, e, N, K, G, n, row);
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0, b = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        double p = orc_e4m3_to_double(x8[m * K + k]) * (double)sx[m] * row[k];
+        acc += p;
+        b += fabs(p);
+      }
+      y[m * W + (n - n0)] = acc;
+      if (bound) bound[m * W + (n - n0)] = b;
+    }
+  }
+  free(row);
+  return ORC_OK;
+}
+
+/* Individual outputs (ms[i], ns[i]) of the W4A8-FP8 layer. */
+int orc_fp8_linear_entries(const uint8_t* x8, const float* sx, int64_t M, const uint32_t* qweight,
+                           const uint16_t* scales, const uint8_t* zeros, const int8_t* e, int64_t N, int64_t K,
+                           int G, const int64_t* ms, const int64_t* ns, int64_t count, double* y, double* bound) {
+  if (M < 0 || bad_shape(N, K, G) || word_in_row(0, G) < 0) return ORC_ERR_SHAPE;
+  double* row = (double*)malloc(sizeof(double) * (size_t)K);
+  int64_t cached = -1;
+  for (int64_t i = 0; i < count; ++i) {
+    int64_t m = ms[i], n = ns[i];
+    if (m < 0 || m >= M || n < 0 || n >= N) { free(row); return ORC_ERR_SHAPE; }
+    if (n != cached) { fp8_row(qweight, scales, zeros, e, N, K, G, n, row); cached = n; }
+    double acc = 0.0, b = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+      double p = orc_e4m3_to_double(x8[m * K + k]) * (double)sx[m] * row[k];
       acc += p;
       b += fabs(p);
     }
