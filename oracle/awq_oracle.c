@@ -366,7 +366,11 @@ int orc_linear_entries(const uint16_t* x, int64_t M, const uint32_t* qweight, co
  *     largest finite E4M3 value); a row of zeros gives sx = 0 and x8 = 0.
  *   - weights: per output channel n, S_n = max over its groups of s, and e[n]
  *     the largest integer with 15 * S_n * 2^e <= 448 (every |q - z| <= 15, so
- *     W^ * 2^e stays within the E4M3 range); W8[n,k] = e4m3(W^[n,k] * 2^e[n]).
+ *     the scaled weights stay within the E4M3 range). With the scale moved by
+ *     that power of two, s' = fp16_rne(s * 2^e[n]) (exact unless it falls
+ *     below the fp16 normal range), W8[n,k] = e4m3(fp16_rne((q - z) * s')).
+ *     Wherever W^ = fp16_rne((q - z) s) is an fp16 normal number this is
+ *     e4m3(W^ * 2^e[n]): scaling by a power of two commutes with rounding.
  *   - y[m,n] = sum_k (x8[m,k] sx[m]) (W8[n,k] 2^-e[n]), here in fp64.
  * e4m3(v) rounds v to the nearest E4M3 value, ties to even, and saturates:
  * |v| >= 448 (or infinite) gives +-448; NaN gives 0x7F.
@@ -454,24 +458,30 @@ int orc_fp8_row_exponents(const uint16_t* scales, int64_t N, int64_t K, int G, i
   return ORC_OK;
 }
 
+/* E4M3 code of weight (n, k), from the packed buffers. */
+static uint8_t fp8_weight(const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros, const int8_t* e,
+                          int64_t N, int64_t K, int G, int64_t n, int64_t k) {
+  int64_t g = k / G;
+  uint32_t q = (qweight[word_index(n, k, K, N, G)] >> nibble_shift((int)(k % 8))) & 0xF;
+  uint32_t z = (zeros[g * (N / 2) + n / 2] >> (4 * (n % 2))) & 0xF;
+  double s2 = orc_half_to_double(orc_double_to_half(ldexp(orc_half_to_double(scales[g * N + n]), e[n])));
+  return orc_double_to_e4m3(orc_half_to_double(orc_double_to_half(((double)q - (double)z) * s2)));
+}
+
 /* W8 [N][K] E4M3 codes of the packed weight scaled by 2^e[n]. */
 int orc_fp8_weights(const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros, const int8_t* e,
                     int64_t N, int64_t K, int G, uint8_t* w8) {
   if (bad_shape(N, K, G) || word_in_row(0, G) < 0) return ORC_ERR_SHAPE;
-  double* row = (double*)malloc(sizeof(double) * (size_t)K);
-  for (int64_t n = 0; n < N; ++n) {
-    packed_row(qweight, scales, zeros, N, K, G, n, row);
-    for (int64_t k = 0; k < K; ++k) w8[n * K + k] = orc_double_to_e4m3(ldexp(row[k], e[n]));
-  }
-  free(row);
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) w8[n * K + k] = fp8_weight(qweight, scales, zeros, e, N, K, G, n, k);
   return ORC_OK;
 }
 
 /* Row n of the W4A8-FP8 weight as the values it stands for: W8[n,k] 2^-e[n]. */
 static void fp8_row(const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros, const int8_t* e,
                     int64_t N, int64_t K, int G, int64_t n, double* row) {
-  packed_row(qweight, scales, zeros, N, K, G, n, row);
-  for (int64_t k = 0; k < K; ++k) row[k] = ldexp(orc_e4m3_to_double(orc_double_to_e4m3(ldexp(row[k], e[n]))), -e[n]);
+  for (int64_t k = 0; k < K; ++k)
+    row[k] = ldexp(orc_e4m3_to_double(fp8_weight(qweight, scales, zeros, e, N, K, G, n, k)), -e[n]);
 }
 
 /* y, bound [M][n1-n0]: output channels n0..n1-1 of the W4A8-FP8 layer, from

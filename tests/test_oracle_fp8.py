@@ -157,8 +157,11 @@ def test_weights_are_the_rounded_scaled_dequant_and_one_hot_reads_them():
     q, z, s = oracle.unpack(qw, sc, ze, N, K)
     wh = oracle.dequant(q, z, s).astype(np.float64)
     scaled = wh * (2.0 ** e.astype(np.float64))[:, None]
-    assert np.abs(scaled).max() <= 448 * (1 + 2.0 ** -11)
-    assert (w8 == _torch_e4m3(np.clip(scaled, -448, 448))).all()
+    assert np.abs(scaled).max() <= 448
+    # where W^ is an fp16 normal number (here: all nonzero weights), W8 is
+    # torch's E4M3 rounding of W^ 2^e
+    assert (np.abs(wh[wh != 0]) >= 2.0 ** -14).all()
+    assert (w8 == _torch_e4m3(scaled)).all()
     x = np.zeros((2, K), np.float16)
     x[0, 7], x[1, 200] = 448.0, -896.0     # sx = 1 and 2 exactly, x8 = +-448
     x8, sx = oracle.fp8_quantize_x(x)
@@ -166,3 +169,22 @@ def test_weights_are_the_rounded_scaled_dequant_and_one_hot_reads_them():
     y, _ = oracle.fp8_linear(x8, sx, qw, sc, ze, e, N, K)
     assert np.array_equal(y[0], 448.0 * _decode(w8[:, 7]) * 2.0 ** -e.astype(np.float64))
     assert np.array_equal(y[1], -896.0 * _decode(w8[:, 200]) * 2.0 ** -e.astype(np.float64))
+
+
+def test_weights_of_groups_with_fp16_subnormal_dequant_values():
+    # scales below 2^-14 / 15 make W^ an fp16 subnormal; the scale is moved by
+    # 2^e before the product is rounded, so W8 keeps full precision there
+    N, K = 16, 256
+    q = np.random.default_rng(5).integers(0, 16, (N, K)).astype(np.uint8)
+    z = np.full((N, K // 128), 7, np.uint8)
+    s = np.full((N, K // 128), 2.0 ** -20 * 1.3, np.float16)
+    s[:, 1] = np.float16(2.0 ** -21 * 1.7)
+    qw, sc, ze = oracle.pack(q, z, s)
+    e = oracle.fp8_row_exponents(sc, N, K)
+    w8 = oracle.fp8_weights(qw, sc, ze, e, N, K)
+    for n in range(N):
+        for k in (0, 5, 127, 128, 200, 255):
+            g = k // 128
+            s2 = np.float64(np.float16(np.float64(s[n, g]) * 2.0 ** int(e[n])))
+            v = np.float64(np.float16((int(q[n, k]) - int(z[n, g])) * s2))
+            assert w8[n, k] == _torch_e4m3(np.array([v]))[0]
