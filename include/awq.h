@@ -154,6 +154,52 @@ awq_status awq_linear(const void* x, const void* qweight, const void* scales, co
                       int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,
                       void* stream);
 
+/* ---------------------------------------------------------------------------
+ * W4A8-FP8 variant of the prefill GEMM
+ * ---------------------------------------------------------------------------
+ * The TensorRT-LLM news item on INT4 AWQ on one H200 says its AWQ kernels
+ * compute in FP8 on the tensor cores; the pages print no recipe. This variant
+ * keeps the packed 4-bit weights of awq_pack unchanged and runs the MMA on
+ * E4M3 (OCP 8-bit floating point, 4 exponent bits, bias 7, 3 fraction bits,
+ * largest finite value 448) with fp32 accumulation:
+ *   sx[m]   = fp32(max_k |x[m][k]|) / 448                (IEEE fp32 division)
+ *   x8[m,k] = e4m3(x[m][k] / sx[m])                      (0 when sx[m] == 0)
+ *   e[n]    = the largest integer with 15 * max_g s[n,g] * 2^e <= 448
+ *   W8[n,k] = e4m3(fp16((q - z) * fp16(s * 2^e[n])))
+ *   y[m][n] = fp16(sum_k x8[m,k] W8[n,k] * sx[m] * 2^-e[n])
+ * e4m3() rounds to the nearest E4M3 value, ties to even, saturating at +-448.
+ * It is a lossy variant: x and the weights each keep 4 significant bits, so y
+ * differs from awq_w4a16_gemm by up to about 2^-3 of sum_k |x W^| (2^-4 from
+ * each operand). Typical use per weight: awq_fp8_row_exponents once (offline,
+ * like awq_pack); per batch: awq_fp8_quantize_x, then awq_w4a8_gemm. */
+
+/* e[n] (int8, one per output channel) from the packed scales fp16 [K/group][N]
+ * as awq_pack wrote them (positive). Shapes and group as for every entry
+ * point; scales 16-byte aligned; e_out any alignment, not overlapping scales. */
+awq_status awq_fp8_row_exponents(const void* scales, int64_t K, int64_t N, int group, void* e_out, void* stream);
+
+/* x fp16 [M][K] -> x8 E4M3 codes uint8 [M][K] and sx fp32 [M] (formulas above).
+ * K % 128 == 0; M >= 0 (0 is a no-op); x, x8 and sx 16-byte aligned and not
+ * overlapping. A row holding inf or NaN gives codes and sx that are not
+ * finite numbers (NaN, or 0 codes with sx = inf). */
+awq_status awq_fp8_quantize_x(const void* x, int64_t M, int64_t K, void* x8, void* sx, void* stream);
+
+/* W8 uint8 [N][K] = the E4M3 codes the W4A8 GEMM multiplies (test surface,
+ * like awq_dequant): row_exp is e from awq_fp8_row_exponents. */
+awq_status awq_dequant_fp8(const void* qweight, const void* scales, const void* zeros, const void* row_exp,
+                           int64_t K, int64_t N, int group, void* w8_out, void* stream);
+
+/* y fp16 [M][N] from x8 [M][K] and sx [M] (awq_fp8_quantize_x), the packed
+ * weight and row_exp [N] (awq_fp8_row_exponents): tcgen05.mma kind::f8f6f4
+ * on E4M3 operands, fp32 accumulation in tensor memory, the weights
+ * dequantized to E4M3 in shared memory just ahead of the MMA. Any M >= 0.
+ * x8, sx, y, the packed buffers and the workspace 16-byte aligned; y must not
+ * overlap any input. The workspace needs only its status word
+ * (ws_bytes >= 256); an expired bounded wait records AWQ_ERR_TIMEOUT there. */
+awq_status awq_w4a8_gemm(const void* x8, const void* sx, const void* qweight, const void* scales, const void* zeros,
+                         const void* row_exp, void* y, int64_t M, int64_t K, int64_t N, int group, void* workspace,
+                         size_t ws_bytes, void* stream);
+
 /* The M at and below which awq_linear takes the GEMV path. */
 int awq_linear_gemv_limit(void);
 

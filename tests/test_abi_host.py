@@ -138,3 +138,38 @@ def test_bounded_wait_self_test_argument_errors():
     assert L.awq_check_bounded_wait(FAKE, 256, 2000000, None) == awq.AWQ_ERR_INVALID_ARG
     assert L.awq_check_bounded_wait(FAKE + 4, 256, 1000, None) == awq.AWQ_ERR_ALIGNMENT
     assert L.awq_check_bounded_wait(FAKE, 16, 1000, None) == awq.AWQ_ERR_WORKSPACE
+
+
+def test_fp8_entry_points_reject_bad_arguments():
+    # awq_fp8_row_exponents(scales, K, N, group, e_out, stream)
+    assert L.awq_fp8_row_exponents(FAKE, 100, 16, 128, FAKE2, None) == awq.AWQ_ERR_SHAPE
+    assert L.awq_fp8_row_exponents(FAKE, 128, 16, 96, FAKE2, None) == awq.AWQ_ERR_UNSUPPORTED
+    assert L.awq_fp8_row_exponents(None, 128, 16, 128, FAKE2, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_fp8_row_exponents(FAKE + 2, 128, 16, 128, FAKE2, None) == awq.AWQ_ERR_ALIGNMENT
+    assert L.awq_fp8_row_exponents(FAKE, 128, 16, 128, FAKE + 4, None) == awq.AWQ_ERR_INVALID_ARG  # overlap
+    # awq_fp8_quantize_x(x, M, K, x8, sx, stream)
+    assert L.awq_fp8_quantize_x(FAKE, 4, 100, FAKE2, FAKE3, None) == awq.AWQ_ERR_SHAPE
+    assert L.awq_fp8_quantize_x(FAKE, -1, 128, FAKE2, FAKE3, None) == awq.AWQ_ERR_SHAPE
+    assert L.awq_fp8_quantize_x(None, 0, 128, None, None, None) == awq.AWQ_OK          # empty batch
+    assert L.awq_fp8_quantize_x(FAKE, 4, 128, None, FAKE3, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_fp8_quantize_x(FAKE, 4, 128, FAKE2 + 8, FAKE3, None) == awq.AWQ_ERR_ALIGNMENT
+    assert L.awq_fp8_quantize_x(FAKE, 4, 128, FAKE + 256, FAKE3, None) == awq.AWQ_ERR_INVALID_ARG  # x8 inside x
+    # awq_dequant_fp8(qweight, scales, zeros, row_exp, K, N, group, w8_out, stream)
+    assert L.awq_dequant_fp8(FAKE, FAKE2, FAKE3, FAKE4, 128, 15, 128, FAKE5, None) == awq.AWQ_ERR_SHAPE
+    assert L.awq_dequant_fp8(FAKE, FAKE2, FAKE3, None, 128, 16, 128, FAKE5, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_dequant_fp8(FAKE, FAKE2, FAKE3, FAKE4, 128, 16, 128, FAKE5 + 1, None) == awq.AWQ_ERR_ALIGNMENT
+    # awq_w4a8_gemm(x8, sx, qweight, scales, zeros, row_exp, y, M, K, N, group, ws, ws_bytes, stream)
+    args = [FAKE, FAKE2, FAKE3, FAKE4, FAKE5, FAKE6, FAKE6 + (1 << 20)]
+    assert L.awq_w4a8_gemm(*args, 8, 128, 16, 128, FAKE6 + (1 << 24), 16, None) == awq.AWQ_ERR_WORKSPACE
+    assert L.awq_w4a8_gemm(*args, -1, 128, 16, 128, FAKE6 + (1 << 24), 256, None) == awq.AWQ_ERR_SHAPE
+    assert L.awq_w4a8_gemm(*args, 8, 128, 16, 256, FAKE6 + (1 << 24), 256, None) == awq.AWQ_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[5] = None
+    assert L.awq_w4a8_gemm(*bad, 8, 128, 16, 128, FAKE6 + (1 << 24), 256, None) == awq.AWQ_ERR_INVALID_ARG
+    bad = list(args)
+    bad[1] = FAKE2 + 4
+    assert L.awq_w4a8_gemm(*bad, 8, 128, 16, 128, FAKE6 + (1 << 24), 256, None) == awq.AWQ_ERR_ALIGNMENT
+    bad = list(args)
+    bad[6] = FAKE                                    # y on top of x8
+    assert L.awq_w4a8_gemm(*bad, 8, 128, 16, 128, FAKE6 + (1 << 24), 256, None) == awq.AWQ_ERR_INVALID_ARG
+    assert L.awq_w4a8_gemm(*args, 0, 128, 16, 128, FAKE6 + (1 << 24), 256, None) == awq.AWQ_OK  # empty batch

@@ -10,7 +10,9 @@ Functions (same names as the C entry points):
   awq_packed_size, awq_workspace_bytes, awq_workspace_init, awq_pack,
   awq_dequant, awq_w4a16_gemv, awq_w4a16_gemm, awq_linear,
   awq_linear_gemv_limit, awq_linear_launches, awq_check_bounded_wait,
-  awq_get_status, awq_status_string, awq_w4a16_gemv_no_alloc.
+  awq_get_status, awq_status_string, awq_w4a16_gemv_no_alloc, and the W4A8-FP8
+  variant awq_fp8_row_exponents, awq_fp8_quantize_x, awq_dequant_fp8,
+  awq_w4a8_gemm.
 """
 from __future__ import annotations
 
@@ -34,7 +36,8 @@ globals().update({name: code for code, name in STATUS_NAMES.items()})
 # Every symbol include/awq.h declares.
 EXPORTS = ("awq_packed_size", "awq_workspace_bytes", "awq_workspace_init", "awq_pack", "awq_dequant",
            "awq_w4a16_gemv", "awq_w4a16_gemm", "awq_linear", "awq_linear_gemv_limit", "awq_get_status",
-           "awq_status_string", "awq_w4a16_gemv_no_alloc", "awq_linear_launches", "awq_check_bounded_wait")
+           "awq_status_string", "awq_w4a16_gemv_no_alloc", "awq_linear_launches", "awq_check_bounded_wait",
+           "awq_fp8_row_exponents", "awq_fp8_quantize_x", "awq_dequant_fp8", "awq_w4a8_gemm")
 
 
 class AwqError(RuntimeError):
@@ -76,6 +79,10 @@ def _load() -> ctypes.CDLL:
     lib.awq_linear_launches.argtypes = [i64, i64, i64, ci]
     lib.awq_check_bounded_wait.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.awq_get_status.argtypes = [vp, vp]
+    lib.awq_fp8_row_exponents.argtypes = [vp, i64, i64, ci, vp, vp]
+    lib.awq_fp8_quantize_x.argtypes = [vp, i64, i64, vp, vp, vp]
+    lib.awq_dequant_fp8.argtypes = [vp, vp, vp, vp, i64, i64, ci, vp, vp]
+    lib.awq_w4a8_gemm.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, sz, vp]
     lib.awq_status_string.argtypes = [ci]
     lib.awq_status_string.restype = ctypes.c_char_p
     for f in EXPORTS:
@@ -196,6 +203,50 @@ def awq_w4a16_gemv_no_alloc(x, qweight, scales, zeros, N, group: int = GROUP, y=
                                        _dev(scales, torch.float16, "scales"), _dev(zeros, torch.uint8, "zeros"),
                                        _dev(y, torch.float16, "y"), M, K, N, group, _stream(x)),
            "awq_w4a16_gemv_no_alloc")
+    return y
+
+
+def awq_fp8_row_exponents(scales: torch.Tensor, K: int, N: int, group: int = GROUP) -> torch.Tensor:
+    """int8 [N]: per output channel, the power of two that moves its weights into
+    the E4M3 range (W4A8-FP8 variant; once per weight, like awq_pack)."""
+    e = torch.empty(N, dtype=torch.int8, device=scales.device)
+    _check(lib.awq_fp8_row_exponents(_dev(scales, torch.float16, "scales"), K, N, group, e.data_ptr(),
+                                     _stream(scales)), "awq_fp8_row_exponents")
+    return e
+
+
+def awq_fp8_quantize_x(x: torch.Tensor):
+    """x fp16 [M][K] -> (x8 uint8 E4M3 codes [M][K], sx float32 [M])."""
+    M, K = x.shape
+    x8 = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib.awq_fp8_quantize_x(_dev(x, torch.float16, "x"), M, K, x8.data_ptr(), sx.data_ptr(), _stream(x)),
+           "awq_fp8_quantize_x")
+    return x8, sx
+
+
+def awq_dequant_fp8(qweight, scales, zeros, row_exp, K: int, N: int, group: int = GROUP) -> torch.Tensor:
+    """uint8 [N][K]: the E4M3 weight codes the W4A8 GEMM multiplies (test surface)."""
+    w8 = torch.empty((N, K), dtype=torch.uint8, device=qweight.device)
+    _check(lib.awq_dequant_fp8(_dev(qweight, torch.int32, "qweight"), _dev(scales, torch.float16, "scales"),
+                               _dev(zeros, torch.uint8, "zeros"), _dev(row_exp, torch.int8, "row_exp"), K, N, group,
+                               w8.data_ptr(), _stream(qweight)), "awq_dequant_fp8")
+    return w8
+
+
+def awq_w4a8_gemm(x8, sx, qweight, scales, zeros, row_exp, N, workspace, group: int = GROUP, y=None):
+    """W4A8-FP8 prefill GEMM (tcgen05 kind::f8f6f4): y fp16 [M][N] from the
+    outputs of awq_fp8_quantize_x and awq_fp8_row_exponents."""
+    M, K = x8.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=x8.device)
+    elif y.shape != (M, N):
+        raise ValueError(f"y must be [{M}, {N}]")
+    _check(lib.awq_w4a8_gemm(_dev(x8, torch.uint8, "x8"), _dev(sx, torch.float32, "sx"),
+                             _dev(qweight, torch.int32, "qweight"), _dev(scales, torch.float16, "scales"),
+                             _dev(zeros, torch.uint8, "zeros"), _dev(row_exp, torch.int8, "row_exp"),
+                             _dev(y, torch.float16, "y"), M, K, N, group, _dev(workspace, torch.uint8, "workspace"),
+                             workspace.numel(), _stream(x8)), "awq_w4a8_gemm")
     return y
 
 

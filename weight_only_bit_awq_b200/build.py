@@ -21,7 +21,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
 # The pack kernel must not contract fp64 operations (bit-exact quantization).
 PER_FILE = {"pack.cu": ["--fmad=false"]}
-SOURCES = ["abi.cu", "pack.cu", "gemv.cu", "gemm_tc.cu", "no_alloc.cu"]
+SOURCES = ["abi.cu", "pack.cu", "gemv.cu", "gemm_tc.cu", "gemm_fp8.cu", "no_alloc.cu"]
 HEADERS = ["awq_internal.cuh", "sm100_ptx.cuh"]
 
 

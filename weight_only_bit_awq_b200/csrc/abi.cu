@@ -241,6 +241,80 @@ awq_status awq_linear(const void* x, const void* qweight, const void* scales, co
 
 int awq_linear_gemv_limit(void) { return g_gemv_limit; }
 
+awq_status awq_fp8_row_exponents(const void* scales, int64_t K, int64_t N, int group, void* e_out, void* stream) {
+  awq_status st = check_kn(K, N, group);
+  if (st != AWQ_OK) return st;
+  if (!scales || !e_out) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(scales)) return AWQ_ERR_ALIGNMENT;
+  if (overlap(e_out, (size_t)N, scales, (size_t)(K / group) * N * 2)) return AWQ_ERR_INVALID_ARG;
+  if ((st = check_device()) != AWQ_OK) return st;
+  cudaError_t e = launch_fp8_row_exponents(static_cast<const __half*>(scales), K, N, group,
+                                           static_cast<int8_t*>(e_out), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+awq_status awq_fp8_quantize_x(const void* x, int64_t M, int64_t K, void* x8, void* sx, void* stream) {
+  if (M < 0 || K <= 0) return AWQ_ERR_SHAPE;
+  if (K % kKPerBlock != 0) return AWQ_ERR_SHAPE;
+  if (K > kMaxK || M > kMaxM) return AWQ_ERR_UNSUPPORTED;
+  if (M == 0) return AWQ_OK;
+  if (!x || !x8 || !sx) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x8) || !aligned16(sx)) return AWQ_ERR_ALIGNMENT;
+  const size_t xb = (size_t)M * K * 2, x8b = (size_t)M * K, sxb = (size_t)M * 4;
+  if (overlap(x, xb, x8, x8b) || overlap(x, xb, sx, sxb) || overlap(x8, x8b, sx, sxb)) return AWQ_ERR_INVALID_ARG;
+  awq_status st = check_device();
+  if (st != AWQ_OK) return st;
+  cudaError_t e = launch_fp8_quantize_x(static_cast<const __half*>(x), M, K, static_cast<uint8_t*>(x8),
+                                        static_cast<float*>(sx), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+awq_status awq_dequant_fp8(const void* qweight, const void* scales, const void* zeros, const void* row_exp,
+                           int64_t K, int64_t N, int group, void* w8_out, void* stream) {
+  awq_status st = check_kn(K, N, group);
+  if (st != AWQ_OK) return st;
+  if (!w8_out || !qweight || !scales || !zeros || !row_exp) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(w8_out) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros)) return AWQ_ERR_ALIGNMENT;
+  const size_t wb = (size_t)K * N, ng = (size_t)(K / group);
+  if (overlap(w8_out, wb, qweight, (size_t)K * N / 2) || overlap(w8_out, wb, scales, ng * N * 2) ||
+      overlap(w8_out, wb, zeros, ng * N / 2) || overlap(w8_out, wb, row_exp, (size_t)N))
+    return AWQ_ERR_INVALID_ARG;
+  if ((st = check_device()) != AWQ_OK) return st;
+  cudaError_t e = launch_dequant_fp8(static_cast<const uint32_t*>(qweight), static_cast<const __half*>(scales),
+                                     static_cast<const uint8_t*>(zeros), static_cast<const int8_t*>(row_exp), K, N,
+                                     group, static_cast<uint8_t*>(w8_out), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+awq_status awq_w4a8_gemm(const void* x8, const void* sx, const void* qweight, const void* scales, const void* zeros,
+                         const void* row_exp, void* y, int64_t M, int64_t K, int64_t N, int group, void* workspace,
+                         size_t ws_bytes, void* stream) {
+  if (M < 0) return AWQ_ERR_SHAPE;
+  awq_status st = check_kn(K, N, group);
+  if (st != AWQ_OK) return st;
+  if (M > kMaxM) return AWQ_ERR_UNSUPPORTED;
+  if ((M > 0 && (!x8 || !sx || !y)) || !qweight || !scales || !zeros || !row_exp || !workspace)
+    return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(x8) || !aligned16(sx) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
+      !aligned16(y) || !aligned16(workspace))
+    return AWQ_ERR_ALIGNMENT;
+  const size_t ybytes = (size_t)M * N * 2, ng = (size_t)(K / group);
+  if (overlap(y, ybytes, x8, (size_t)M * K) || overlap(y, ybytes, sx, (size_t)M * 4) ||
+      overlap(y, ybytes, qweight, (size_t)K * N / 2) || overlap(y, ybytes, scales, ng * N * 2) ||
+      overlap(y, ybytes, zeros, ng * N / 2) || overlap(y, ybytes, row_exp, (size_t)N) ||
+      overlap(y, ybytes, workspace, ws_bytes))
+    return AWQ_ERR_INVALID_ARG;
+  if (ws_bytes < kWsHeaderBytes) return AWQ_ERR_WORKSPACE;
+  if (M == 0) return AWQ_OK;
+  if ((st = check_device()) != AWQ_OK) return st;
+  cudaError_t e = launch_gemm_fp8(static_cast<const uint8_t*>(x8), static_cast<const float*>(sx),
+                                  static_cast<const uint32_t*>(qweight), static_cast<const __half*>(scales),
+                                  static_cast<const uint8_t*>(zeros), static_cast<const int8_t*>(row_exp),
+                                  static_cast<__half*>(y), M, K, N, group, status_word(workspace),
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group) {
   if (M <= 0 || M > kMaxM || check_kn(K, N, group) != AWQ_OK) return 0;
   if (M > g_gemv_limit) return 1;

@@ -85,6 +85,18 @@ cudaError_t launch_gemm(const __half* x, const uint32_t* qweight, const __half* 
                         __half* y, int64_t M, int64_t K, int64_t N, int group, uint32_t* status,
                         cudaStream_t stream);
 
+// W4A8-FP8 variant (gemm_fp8.cu).
+cudaError_t launch_fp8_row_exponents(const __half* scales, int64_t K, int64_t N, int group, int8_t* e_out,
+                                     cudaStream_t stream);
+cudaError_t launch_fp8_quantize_x(const __half* x, int64_t M, int64_t K, uint8_t* x8, float* sx,
+                                  cudaStream_t stream);
+cudaError_t launch_dequant_fp8(const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
+                               const int8_t* row_exp, int64_t K, int64_t N, int group, uint8_t* w8_out,
+                               cudaStream_t stream);
+cudaError_t launch_gemm_fp8(const uint8_t* x8, const float* sx, const uint32_t* qweight, const __half* scales,
+                            const uint8_t* zeros, const int8_t* row_exp, __half* y, int64_t M, int64_t K, int64_t N,
+                            int group, uint32_t* status, cudaStream_t stream);
+
 // Packed word order inside a row's 128-input block, for group size G (128, 64
 // or 32): word w = 4t + j holds the eight inputs from k0(w) = G (j / J) +
 // 8 (t J + j % J), J = G / 32 (for G = 128 simply 8w). The four words with the
