@@ -21,7 +21,9 @@
 // BN-token tile per CTA, warp 0 loads x8 by TMA (one 128-byte-wide box per
 // 128-input k-block, 128-byte swizzle), warp 1 issues 4 MMAs of K = 32 per
 // k-block, warp 2 copies the packed codes and the tile's scale and zero rows,
-// warps 3-6 dequantize (thread = weight row) and then run the epilogue. Every
+// warps 3-10 dequantize (two threads per weight row, half of its codes each:
+// two warps per SM sub-partition hide the conversion latency) and then run the
+// epilogue (warps w and w + 4 share TMEM lanes and split the columns). Every
 // mbarrier wait is bounded; on expiry AWQ_ERR_TIMEOUT goes to the status word
 // and the CTA drains and exits.
 #include <cuda_fp8.h>
@@ -197,7 +199,7 @@ constexpr int kQBytes = 8 * 1024;
 constexpr int kQScaleOff = kQBytes, kQZeroOff = kQScaleOff + 4 * 256;
 constexpr int kQStride = kQZeroOff + 4 * 64;
 constexpr int kWBytes = kBM * kKPerBlock;  // 16 KiB: 128 rows x 128 E4M3 weights
-constexpr int kWarpX = 0, kWarpMma = 1, kWarpQ = 2, kFirstDeqWarp = 3, kNumDeqWarps = 4;
+constexpr int kWarpX = 0, kWarpMma = 1, kWarpQ = 2, kFirstDeqWarp = 3, kNumDeqWarps = 8;
 constexpr int kDeqThreads = kNumDeqWarps * 32;
 constexpr int kThreads = (kFirstDeqWarp + kNumDeqWarps) * 32;
 
@@ -346,8 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ---------------- dequantize to E4M3, then epilogue ----------------
-    const int row = threadIdx.x - kFirstDeqWarp * 32;  // 0..127, row & 31 == lane
-    const int rot = (lane >> 1) & 3;  // chunk rotation: conflict-free shared loads
+    // Thread d = (row, half): row = d / 2 takes codes words 8 half .. 8 half + 7
+    // of its row (two 16-byte chunks, read in a rotated order so that the
+    // warp's shared loads are bank-conflict free).
+    const int d = threadIdx.x - kFirstDeqWarp * 32;  // 0..255
+    const int row = d >> 1, hf = d & 1;
+    const int rot = (row >> 1) & 1;
     constexpr int kGPK = kKPerBlock / GS;
     const int nn = n0 + row;
     const int e = nn < N ? row_exp[nn] : 0;
@@ -357,10 +363,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qs = kb % kQStages;
       if (!(ok = wait_bar(bar(kBarQFull + qs), (kb / kQStages) & 1, abort_flag, status))) break;
       const uint8_t* qst = smem + L::kQOff + qs * kQStride;
-      const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64;
-      uint4 c[4];
+      const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64 + 32 * hf;
+      uint4 c[2];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 3));
+      for (int jj = 0; jj < 2; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 1));
       // scale and zero point of this row, per group (rows past N read stale
       // values: their outputs are never stored)
       uint32_t sb[kGPK], z[kGPK];
@@ -378,8 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 0; g < kGPK; ++g) gc[g] = group_consts(sb[g], z[g], pow2e);
       uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int cj = (jj + rot) & 3;  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
+      for (int jj = 0; jj < 2; ++jj) {
+        const int cj = 2 * hf + ((jj + rot) & 1);  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
         const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
 #pragma unroll
         for (int ww = 0; ww < 4; ++ww) {
@@ -396,12 +402,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && wait_bar(bar(kBarAcc), 0, abort_flag, status)) {
       ptx::tc_fence_after();
-      const int quad = warp & 3;  // this warp may read TMEM lanes 32*quad .. +31
+      const int quad = warp & 3;                          // this warp may read TMEM lanes 32*quad .. +31
+      const int colh = (warp - kFirstDeqWarp) >> 2;       // and takes half of the columns
       const int r = 32 * quad + lane;
       const int n = n0 + r;
       const float pow2ne = pow2f(-(n < N ? row_exp[n] : 0));
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = colh * (BN / 2); c0 < (colh + 1) * (BN / 2); c0 += 32) {
         if (m0 + c0 >= M) break;
         uint32_t v[32];
         ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)c0, v);
