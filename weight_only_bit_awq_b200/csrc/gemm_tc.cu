@@ -10,19 +10,21 @@
 // operand A) x BN tokens (operand B, BN = 128 or 256) x the whole K, one tile
 // per CTA. Accumulation in tensor memory (fp32, BN columns x 128 lanes).
 //
-// Warp roles (224 threads):
+// Warp roles (352 threads):
 //   warp 0  lane 0 issues TMA loads of x: 64-k x BN boxes with the 128-byte
 //           swizzle, exactly the K-major operand layout tcgen05 reads.
 //   warp 1  allocates tensor memory; lane 0 issues tcgen05.mma (4 per 64-k
 //           stage, K = 16 each) and commits to the stage barriers.
 //   warp 2  lane 0 issues bulk copies of the packed weight: the tile's 8 row
 //           blocks of one 128-k block are one contiguous 8 KiB run.
-//   warps 3-6 dequantize: thread r owns weight row r of the tile, reads its
-//           64 B of codes for the k-block from shared memory, forms
-//           fp16_rne((q - z) * s) (the exact value the dequant kernel and the
-//           CPU oracle produce) and stores it, swizzled, into the A-operand
-//           buffer; afterwards they drain the accumulator (tcgen05.ld) and
-//           write fp16 y.
+//   warps 3-10 dequantize: threads 2r and 2r + 1 own weight row r of the
+//           tile, each reads half of its 64 B of codes for the k-block from
+//           shared memory, forms fp16_rne((q - z) * s) (the exact value the
+//           dequant kernel and the CPU oracle produce) and stores it,
+//           swizzled, into the A-operand buffer (two warps per SM
+//           sub-partition hide the dependent fp16 chains); afterwards they
+//           drain the accumulator (tcgen05.ld; warps w and w + 4 share TMEM
+//           lanes and split the columns) and write fp16 y.
 // Rings: x 4 x (BN x 64 k), dequantized weight 2 x (128 x 128 k), packed
 // weight 3 x 8 KiB, each with full/empty mbarriers. Every wait is bounded
 // (2 s of %globaltimer); on expiry the CTA records AWQ_ERR_TIMEOUT in the
@@ -49,7 +51,7 @@ constexpr int kQScaleOff = kQBytes, kQZeroOff = kQScaleOff + 4 * 256;
 constexpr int kQStride = kQZeroOff + 4 * 64;
 constexpr int kWHalfBytes = kBM * 64 * 2;  // 16 KiB: 128 rows x 64 k
 constexpr int kWBytes = 2 * kWHalfBytes;
-constexpr int kWarpX = 0, kWarpMma = 1, kWarpQ = 2, kFirstDeqWarp = 3, kNumDeqWarps = 4;
+constexpr int kWarpX = 0, kWarpMma = 1, kWarpQ = 2, kFirstDeqWarp = 3, kNumDeqWarps = 8;
 constexpr int kDeqThreads = kNumDeqWarps * 32;
 constexpr int kThreads = (kFirstDeqWarp + kNumDeqWarps) * 32;
 
@@ -234,18 +236,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ---------------- dequantize, then epilogue ----------------
-    const int row = threadIdx.x - kFirstDeqWarp * 32;  // 0..127, row & 31 == lane
-    const int rot = (lane >> 1) & 3;  // chunk rotation: conflict-free shared loads and stores
+    // Thread d = (row, half): row = d / 2 takes words 8 half .. 8 half + 7 of
+    // its row, two 16-byte chunks read and stored in a rotated order (the
+    // rotation also depends on the half) so that every 8-lane phase of the
+    // shared loads and of the swizzled stores touches distinct banks.
+    const int d = threadIdx.x - kFirstDeqWarp * 32;  // 0..255
+    const int row = d >> 1, hf = d & 1;
+    const int rot = ((row >> 1) ^ hf) & 1;
     constexpr int kGPK = kKPerBlock / GS;
     bool ok = true;
     for (int kb = 0; kb < KB; ++kb) {
       const int qs = kb % kQStages;
       if (!(ok = wait_bar(bar(kBarQFull + qs), (kb / kQStages) & 1, abort_flag, status))) break;
       const uint8_t* qst = smem + L::kQOff + qs * kQStride;
-      const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64;
-      uint4 c[4];
+      const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64 + 32 * hf;
+      uint4 c[2];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 3));
+      for (int jj = 0; jj < 2; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 1));
       // fp16 bits of the scale and the zero point of this row, per group (rows
       // past N read stale values: their outputs are never stored)
       uint32_t s[kGPK], z[kGPK];
@@ -268,8 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int cj = (jj + rot) & 3;  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
+      for (int jj = 0; jj < 2; ++jj) {
+        const int cj = 2 * hf + ((jj + rot) & 1);  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
         const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
 #pragma unroll
         for (int ww = 0; ww < 4; ++ww) {
@@ -287,20 +294,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && wait_bar(bar(kBarAcc), 0, abort_flag, status)) {
       ptx::tc_fence_after();
-      const int quad = warp & 3;  // this warp may read TMEM lanes 32*quad .. +31
+      const int quad = warp & 3;                     // this warp may read TMEM lanes 32*quad .. +31
+      const int colh = (warp - kFirstDeqWarp) >> 2;  // and takes half of the columns
       const int r = 32 * quad + lane;
       const int nn = n0 + r;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = colh * (BN / 2); c0 < (colh + 1) * (BN / 2); c0 += 32) {
         if (m0 + c0 >= M) break;
         uint32_t v[32];
         ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)c0, v);
         ptx::tmem_wait_ld();
         if (nn < N) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 32; j += 2) {
             const int m = m0 + c0 + j;
-            if (m < M) y[(int64_t)m * N + nn] = __float2half_rn(__uint_as_float(v[j]));
+            // two conversions in one instruction, each rounded to nearest even
+            const __half2 h = __floats2half2_rn(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+            if (m < M) y[(int64_t)m * N + nn] = __low2half(h);
+            if (m + 1 < M) y[(int64_t)(m + 1) * N + nn] = __high2half(h);
           }
         }
       }
