@@ -378,6 +378,38 @@ def run_ours(args):
         tflops = 2.0 * Mp * PL.N * PL.K / (pms * 1e-3) / 1e12
         prefill = {"workload": f"{PREFILL[1]} K={PL.K} N={PL.N} M={Mp}", "ms": pms, "tflops_per_gpu": tflops,
                    "peak_tflops": tc_burst, "frac": tflops / tc_burst, "peak_kind": f"{peak_kind} bf16 burst"}
+        # W4A8-FP8 variant on the same layer: per call, per-token E4M3
+        # quantization of x plus the kind::f8f6f4 GEMM (the row exponents are
+        # per weight, computed once like the packing)
+        e8 = awq.awq_fp8_row_exponents(pq[1], PL.K, PL.N)
+        x8 = torch.empty((Mp, PL.K), dtype=torch.uint8, device=dev)
+        sx = torch.empty(Mp, dtype=torch.float32, device=dev)
+
+        def w4a8_call():
+            awq.lib.awq_fp8_quantize_x(xp.data_ptr(), Mp, PL.K, x8.data_ptr(), sx.data_ptr(), stream.cuda_stream)
+            awq.awq_w4a8_gemm(x8, sx, *pq, e8, PL.N, pws, y=yp)
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                w4a8_call()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            f0.record(stream)
+            for _ in range(reps):
+                w4a8_call()
+            f1.record(stream)
+        torch.cuda.synchronize()
+        st = awq.awq_get_status(pws)
+        if st != awq.AWQ_OK:
+            raise RuntimeError(awq.awq_status_string(st))
+        fms = max_over_ranks(f0.elapsed_time(f1)) / reps
+        ftf = 2.0 * Mp * PL.N * PL.K / (fms * 1e-3) / 1e12
+        prefill["w4a8_fp8"] = {"ms": fms, "tflops_per_gpu": ftf, "peak_tflops": 2 * tc_burst,
+                               "frac": ftf / (2 * tc_burst),
+                               "peak_kind": f"{peak_kind} bf16 burst x 2 (nominal dense fp8 : bf16 = 4.5 : 2.25)",
+                               "includes": "per-token E4M3 quantization of x + tcgen05 kind::f8f6f4 GEMM"}
+        del x8, sx, e8
 
     # ---- comparator: the same layers as dense fp16 weights through cuBLAS ----
     # (torch.nn.functional.linear; a library call, timed the same way: CUDA
@@ -519,6 +551,77 @@ def run_single(args):
     return 0
 
 
+def run_sharded(args):
+    """N-sharded strong scaling of the decode layer set: every rank holds the
+    packed weights of its slice of each layer's output channels (whole groups
+    of 128), runs its GEMVs and all-gathers y (NCCL), so each step produces
+    every layer's full output on every rank. No CUDA graphs (the all-gather
+    is a collective), so a step also pays the host's launch time."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import weight_only_bit_awq_b200 as awq
+    from weight_only_bit_awq_b200.sharding import ShardedLinear
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    wl = awq_synth.WORKLOADS[WORKLOAD]
+    shards, xs = [], []
+    for L in wl.layers:
+        W = torch.from_numpy(awq_synth.layer_weight(0, wl, L).view(np.uint16)).view(torch.float16).to(dev)
+        shards.append(ShardedLinear(W, world, rank))
+        del W
+        xs.append(torch.from_numpy(awq_synth.layer_input(0, wl, L, M_DECODE).view(np.uint16))
+                  .view(torch.float16).to(dev))
+    step_bytes = sum(algo_bytes(M_DECODE, L.K, L.N) for L in wl.layers)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def step():
+        return [sl.forward_full(x) for sl, x in zip(shards, xs)]
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        ys = step()
+    e1.record()
+    barrier()
+    ms = reduce_max(e0.elapsed_time(e1), world, dev)
+    assert all(y.shape == (M_DECODE, L.N) for y, L in zip(ys, wl.layers))
+    st = [awq.awq_get_status(sl.ws) for sl in shards]
+    if any(st):
+        raise RuntimeError(awq.awq_status_string(max(st)))
+    launches = sum(awq.awq_linear_launches(M_DECODE, L.K, sl.n_local) for sl, L in zip(shards, wl.layers))
+    line = {
+        "metric": METRIC, "value": step_bytes * args.steps / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M_DECODE, "group": 128,
+                   "layers": [[L.name, L.K, L.N] for L in wl.layers],
+                   "parallelism": f"N-sharded x{world} (whole groups of 128 channels) + all-gather of y",
+                   "timing": "eager launches, CUDA events, max over ranks"},
+        "gpu_launches": launches * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -532,6 +635,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=60.0, help="seconds of oracle work in the reference arm")
     ap.add_argument("--single", choices=sorted(SINGLE), help="launch one kernel on one layer (profiling target)")
     ap.add_argument("--reps", type=int, default=4)
+    ap.add_argument("--shard", action="store_true",
+                    help="N-shard the decode layers across the ranks (strong scaling) instead of replicas")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -539,6 +644,8 @@ def main():
         return run_reference(args)
     if args.single:
         return run_single(args)
+    if args.shard:
+        return run_sharded(args)
     return run_ours(args)
 
 
