@@ -515,6 +515,7 @@ SINGLE = {
     # one kernel on a layer larger than the 126 MB L2, for profiler captures
     "gemv": ("llama2_70b_decode", "gate_up", 1),     # 235 MB packed weight, M = 1
     "gemm": ("prefill", "llama3_gate_up", 2048),     # 58 MB weight + 16 MB x + 117 MB y
+    "gemm_fp8": ("prefill", "llama3_gate_up", 2048),  # the same layer through the W4A8-FP8 GEMM
 }
 
 
@@ -535,6 +536,12 @@ def run_single(args):
     x = torch.from_numpy(awq_synth.layer_input(0, wl, L, M).view(np.uint16)).view(torch.float16).to(dev)
     y = torch.empty((M, L.N), dtype=torch.float16, device=dev)
     fn = awq.awq_w4a16_gemv if args.single == "gemv" else awq.awq_w4a16_gemm
+    if args.single == "gemm_fp8":
+        e8 = awq.awq_fp8_row_exponents(packed[1], L.K, L.N)
+        x8, sx = awq.awq_fp8_quantize_x(x)
+
+        def fn(x_, qw, sc, ze, N_, ws_, y=None):  # the GEMM alone: x was quantized above
+            return awq.awq_w4a8_gemm(x8, sx, qw, sc, ze, e8, N_, ws_, y=y)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.reps + 1)]
     ev[0].record()
     for i in range(args.reps):
