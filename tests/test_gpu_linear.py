@@ -306,3 +306,34 @@ def test_decode_non_finite_activation_gives_non_finite_outputs(M, bad):
     y = _run(awq.awq_w4a16_gemv, x, dev, N).astype(np.float64)
     assert not np.isfinite(y[M - 1]).any()
     assert np.isfinite(y[:M - 1]).all()
+
+
+# ---- decode at M = 1: more layer shapes ----------------------------------------
+# K of one k-block, a ragged 9, 32 and 86 k-blocks; a last group of 4 row
+# blocks; last groups of a single row block; 172 and 80 groups; K = 8192. Every
+# output against the oracle, and two calls bit for bit equal.
+ROWS_CASES = [(128, 4096), (1152, 4096), (4096, 4096), (11008, 4096), (4096, 2368), (2048, 6160), (4096, 12304),
+              (1024, 22016), (8192, 10240)]
+
+
+@pytest.mark.parametrize("K,N", ROWS_CASES)
+def test_decode_m1_shapes_match_oracle(K, N):
+    W, dev, hp = _packed(N, K, f"rows{K}x{N}")
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"rows{K}x{N}/x"), 1, K, 1.0)
+    y = _run(awq.awq_w4a16_gemv, x, dev, N)
+    y_ref, b = oracle.linear(x, *hp, N, K)
+    check_close(y, y_ref, b, f"rows K={K} N={N}")
+    y2 = _run(awq.awq_w4a16_gemv, x, dev, N)
+    assert (y2.view(np.uint16) == y.view(np.uint16)).all()        # deterministic
+
+
+def test_decode_m1_one_hot_wide_layer_gives_the_dequantized_weight_exactly():
+    K, N = 1024, 4096
+    W, dev, hp = _packed(N, K, "rows_onehot")
+    q, z, s = oracle.unpack(*hp, N, K)
+    wh = oracle.dequant(q, z, s)
+    for k in (0, 127, 128, 555, 1023):
+        x = np.zeros((1, K), np.float16)
+        x[0, k] = 1.0
+        y = _run(awq.awq_w4a16_gemv, x, dev, N)
+        assert (y[0].view(np.uint16) == wh[:, k].view(np.uint16)).all(), k
