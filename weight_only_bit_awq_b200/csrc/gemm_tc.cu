@@ -7,24 +7,28 @@
 // tensor cores. The weights are dequantized just ahead of the MMA.
 //
 // Tile: 128 output channels (the MMA M dimension, "swap AB": the weight is
-// operand A) x BN tokens (operand B, BN = 128 or 256) x the whole K, one tile
-// per CTA. Accumulation in tensor memory (fp32, BN columns x 128 lanes).
+// operand A) x BN tokens (operand B, BN = 128 or 256) x the whole K.
+// Persistent: one CTA per SM walks tiles c, c + P, ...; accumulation in tensor
+// memory in two accumulators (fp32, 2 x BN columns x 128 lanes), so one tile's
+// epilogue overlaps the next tile's main loop, and the rings below run on
+// across tile boundaries (no pipeline refill per tile).
 //
-// Warp roles (352 threads):
+// Warp roles (480 threads):
 //   warp 0  lane 0 issues TMA loads of x: 64-k x BN boxes with the 128-byte
 //           swizzle, exactly the K-major operand layout tcgen05 reads.
 //   warp 1  allocates tensor memory; lane 0 issues tcgen05.mma (4 per 64-k
-//           stage, K = 16 each) and commits to the stage barriers.
-//   warp 2  lane 0 issues bulk copies of the packed weight: the tile's 8 row
-//           blocks of one 128-k block are one contiguous 8 KiB run.
+//           stage, K = 16 each) into the tile's accumulator and commits to the
+//           stage barriers and, at the end of a tile, to its accumulator's.
+//   warp 2  issues bulk copies of the packed weight: the tile's 8 row blocks
+//           of one 128-k block are one contiguous 8 KiB run.
 //   warps 3-10 dequantize: threads 2r and 2r + 1 own weight row r of the
 //           tile, each reads half of its 64 B of codes for the k-block from
 //           shared memory, forms fp16_rne((q - z) * s) (the exact value the
 //           dequant kernel and the CPU oracle produce) and stores it,
 //           swizzled, into the A-operand buffer (two warps per SM
-//           sub-partition hide the dependent fp16 chains); afterwards they
-//           drain the accumulator (tcgen05.ld; warps w and w + 4 share TMEM
-//           lanes and split the columns) and write fp16 y.
+//           sub-partition hide the dependent fp16 chains).
+//   warps 11-14 drain a finished accumulator (tcgen05.ld; warp w reads TMEM
+//           lanes 32 (w % 4) ..) into fp16 y and release it.
 // Rings: x 4 x (BN x 64 k), dequantized weight 2 x (128 x 128 k), packed
 // weight 3 x 8 KiB, each with full/empty mbarriers. Every wait is bounded
 // (2 s of %globaltimer); on expiry the CTA records AWQ_ERR_TIMEOUT in the
@@ -52,14 +56,15 @@ constexpr int kQStride = kQZeroOff + 4 * 64;
 constexpr int kWHalfBytes = kBM * 64 * 2;  // 16 KiB: 128 rows x 64 k
 constexpr int kWBytes = 2 * kWHalfBytes;
 constexpr int kWarpX = 0, kWarpMma = 1, kWarpQ = 2, kFirstDeqWarp = 3, kNumDeqWarps = 8;
-constexpr int kDeqThreads = kNumDeqWarps * 32;
-constexpr int kThreads = (kFirstDeqWarp + kNumDeqWarps) * 32;
+constexpr int kFirstEpiWarp = kFirstDeqWarp + kNumDeqWarps, kNumEpiWarps = 4;
+constexpr int kDeqThreads = kNumDeqWarps * 32, kEpiThreads = kNumEpiWarps * 32;
+constexpr int kThreads = (kFirstEpiWarp + kNumEpiWarps) * 32;
 
 // barrier indices
 constexpr int kBarXFull = 0, kBarXEmpty = kBarXFull + kXStages, kBarWFull = kBarXEmpty + kXStages,
               kBarWEmpty = kBarWFull + kWStages, kBarQFull = kBarWEmpty + kWStages,
-              kBarQEmpty = kBarQFull + kQStages, kBarAcc = kBarQEmpty + kQStages, kBarDrain = kBarAcc + 1,
-              kNumBars = kBarDrain + 1;
+              kBarQEmpty = kBarQFull + kQStages, kBarAccFull = kBarQEmpty + kQStages, kBarAccEmpty = kBarAccFull + 2,
+              kBarDrain = kBarAccEmpty + 2, kNumBars = kBarDrain + 1;
 
 template <int BN>
 struct Layout {
@@ -102,6 +107,11 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, __half2 zlo, __half2 z
 }
 
 // GS: group size (128, 64 or 32), kGPK = 128 / GS groups per k-block.
+// Persistent: CTA c computes tiles c, c + P, c + 2P, ... (P = gridDim.x; tile
+// t is token tile t % MT of channel tile t / MT, so the CTAs running at the
+// same time share a few weight tiles). Every role walks the same tile
+// sequence; the rings run on across tile boundaries, and the two accumulators
+// let the epilogue warps drain tile j while the MMA warp fills tile j + 1.
 template <int BN, int GS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
@@ -116,9 +126,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BN;
-  const int n0 = blockIdx.y * kBM;
   const int KB = K / kKPerBlock;
+  const int MT = (M + BN - 1) / BN, NT = (N + kBM - 1) / kBM, T = MT * NT;
+  const int P = gridDim.x;
+  const int ntiles = blockIdx.x < T ? (T - 1 - (int)blockIdx.x) / P + 1 : 0;  // tiles of this CTA
+  auto tile_m0 = [&](int it) { return ((int)blockIdx.x + it * P) % MT * BN; };
+  auto tile_nt = [&](int it) { return ((int)blockIdx.x + it * P) / MT; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kXStages; ++i) {
@@ -134,7 +147,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(bar(kBarQFull + i), 33);
       ptx::mbar_init(bar(kBarQEmpty + i), kDeqThreads);
     }
-    ptx::mbar_init(bar(kBarAcc), 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(kBarAccFull + i), 1);
+      ptx::mbar_init(bar(kBarAccEmpty + i), kEpiThreads);
+    }
     ptx::mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
@@ -143,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::prefetch_tensormap(&tmap_x);
   }
   if (warp == kWarpMma) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), BN);
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 2 * BN);
     ptx::tmem_relinquish();
     ptx::tc_fence_before();
   }
@@ -152,55 +168,62 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == kWarpX) {
-    // ---------------- x producer ----------------
+    // ---------------- x producer: 2 boxes of 64 k per k-block ----------------
     if (lane == 0) {
-      const int nst = 2 * KB;
-      int i = 0;
-      for (; i < nst; ++i) {
-        const int s = i % kXStages;
-        if (!wait_bar(bar(kBarXEmpty + s), ((i / kXStages) & 1) ^ 1, abort_flag, status)) break;
-        ptx::mbar_arrive_expect_tx(bar(kBarXFull + s), L::kXBytes);
-        ptx::tma_load_2d(sbase + L::kXOff + s * L::kXBytes, &tmap_x, i * 64, m0, bar(kBarXFull + s));
+      int i = 0;  // stage uses so far
+      bool ok = true;
+      for (int it = 0; it < ntiles && ok; ++it) {
+        const int m0 = tile_m0(it);
+        for (int h = 0; h < 2 * KB; ++h, ++i) {
+          const int s = i % kXStages;
+          if (!(ok = wait_bar(bar(kBarXEmpty + s), ((i / kXStages) & 1) ^ 1, abort_flag, status))) break;
+          ptx::mbar_arrive_expect_tx(bar(kBarXFull + s), L::kXBytes);
+          ptx::tma_load_2d(sbase + L::kXOff + s * L::kXBytes, &tmap_x, h * 64, m0, bar(kBarXFull + s));
+        }
       }
-      if (i < nst)  // aborting: let the copies already issued land
+      if (!ok)  // aborting: let the copies already issued land
         for (int j = (i > kXStages ? i - kXStages : 0); j < i; ++j)
           drain_bar(bar(kBarXFull + j % kXStages), (j / kXStages) & 1);
     }
     __syncwarp();
   } else if (warp == kWarpQ) {
     // ---------------- packed-weight producer ----------------
-    // The R <= 8 row blocks of this tile's group are one contiguous run of
+    // The R <= 8 row blocks of a tile's group are one contiguous run of
     // R KiB per k-block in the packed layout: one 1-D bulk copy each. The
     // tile's scale and zero-point rows of the k-block follow by cp.async.
     constexpr int kGPK = kKPerBlock / GS;
-    const int64_t NB = N / kRowsPerBlock, gi = blockIdx.y;
-    const uint32_t qbytes = (uint32_t)(group_rows(gi, NB) * 1024);
-    int kb = 0;
-    for (; kb < KB; ++kb) {
-      const int s = kb % kQStages;
-      bool ok = true;
-      if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((kb / kQStages) & 1) ^ 1, abort_flag, status);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const uint32_t st = sbase + L::kQOff + s * kQStride;
-      if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qbytes);
-      __syncwarp();
-      if (lane == 0)
-        ptx::bulk_g2s(st, qweight + unit_first_block(gi, kb, KB, NB) * kWordsPerBlock, qbytes, bar(kBarQFull + s));
-      for (int p = lane; p < kGPK * 16; p += 32) {  // kGPK rows of 128 scales: 16 B = 8 output channels
-        const int g = p >> 4, l = p & 15;
-        if (n0 + 8 * l < N)
-          ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
+    const int64_t NB = N / kRowsPerBlock;
+    int i = 0;
+    bool ok = true;
+    for (int it = 0; it < ntiles && ok; ++it) {
+      const int64_t gi = tile_nt(it);
+      const int n0 = (int)gi * kBM;
+      const uint32_t qbytes = (uint32_t)(group_rows(gi, NB) * 1024);
+      for (int kb = 0; kb < KB; ++kb, ++i) {
+        const int s = i % kQStages;
+        if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((i / kQStages) & 1) ^ 1, abort_flag, status);
+        if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+        const uint32_t st = sbase + L::kQOff + s * kQStride;
+        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qbytes);
+        __syncwarp();
+        if (lane == 0)
+          ptx::bulk_g2s(st, qweight + unit_first_block(gi, kb, KB, NB) * kWordsPerBlock, qbytes, bar(kBarQFull + s));
+        for (int p = lane; p < kGPK * 16; p += 32) {  // kGPK rows of 128 scales: 16 B = 8 output channels
+          const int g = p >> 4, l = p & 15;
+          if (n0 + 8 * l < N)
+            ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
+        }
+        for (int p = lane; p < kGPK * 8; p += 32) {  // kGPK rows of 64 zero bytes: 8 B = 16 output channels
+          const int g = p >> 3, l = p & 7;
+          if (n0 + 16 * l < N)
+            ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l,
+                            zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
+        }
+        ptx::cp_async_arrive_noinc(bar(kBarQFull + s));
       }
-      for (int p = lane; p < kGPK * 8; p += 32) {  // kGPK rows of 64 zero bytes: 8 B = 16 output channels
-        const int g = p >> 3, l = p & 7;
-        if (n0 + 16 * l < N)
-          ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l,
-                          zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
-      }
-      ptx::cp_async_arrive_noinc(bar(kBarQFull + s));
     }
-    if (kb < KB && lane == 0)
-      for (int j = (kb > kQStages ? kb - kQStages : 0); j < kb; ++j)
+    if (!ok && lane == 0)
+      for (int j = (i > kQStages ? i - kQStages : 0); j < i; ++j)
         drain_bar(bar(kBarQFull + j % kQStages), (j / kQStages) & 1);
     __syncwarp();
   } else if (warp == kWarpMma) {
@@ -208,34 +231,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = ptx::idesc_f16_f32(kBM, BN);
       bool ok = true;
-      for (int kb = 0; kb < KB && ok; ++kb) {
-        const int ws = kb % kWStages;
-        if (!(ok = wait_bar(bar(kBarWFull + ws), (kb / kWStages) & 1, abort_flag, status))) break;
+      int wi = 0, xi = 0;  // W and x stage uses so far
+      for (int it = 0; it < ntiles && ok; ++it) {
+        const int acc = it & 1;
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);  // column offset of this accumulator
+        if (!(ok = wait_bar(bar(kBarAccEmpty + acc), ((it >> 1) & 1) ^ 1, abort_flag, status))) break;
         ptx::tc_fence_after();
-        for (int h = 0; h < 2; ++h) {
-          const int i = 2 * kb + h, s = i % kXStages;
-          if (!(ok = wait_bar(bar(kBarXFull + s), (i / kXStages) & 1, abort_flag, status))) break;
+        for (int kb = 0; kb < KB && ok; ++kb, ++wi) {
+          const int ws = wi % kWStages;
+          if (!(ok = wait_bar(bar(kBarWFull + ws), (wi / kWStages) & 1, abort_flag, status))) break;
           ptx::tc_fence_after();
-          const uint32_t a_base = sbase + L::kWOff + ws * kWBytes + h * kWHalfBytes;
-          const uint32_t b_base = sbase + L::kXOff + s * L::kXBytes;
+          for (int h = 0; h < 2; ++h, ++xi) {
+            const int s = xi % kXStages;
+            if (!(ok = wait_bar(bar(kBarXFull + s), (xi / kXStages) & 1, abort_flag, status))) break;
+            ptx::tc_fence_after();
+            const uint32_t a_base = sbase + L::kWOff + ws * kWBytes + h * kWHalfBytes;
+            const uint32_t b_base = sbase + L::kXOff + s * L::kXBytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            ptx::mma_f16_ss(tmem_base, ptx::desc_kmajor_sw128(a_base + 32 * kk),
-                            ptx::desc_kmajor_sw128(b_base + 32 * kk), idesc, (kb | h | kk) != 0);
-          ptx::mma_commit(bar(kBarXEmpty + s));
+            for (int kk = 0; kk < 4; ++kk)
+              ptx::mma_f16_ss(d_tmem, ptx::desc_kmajor_sw128(a_base + 32 * kk),
+                              ptx::desc_kmajor_sw128(b_base + 32 * kk), idesc, (kb | h | kk) != 0);
+            ptx::mma_commit(bar(kBarXEmpty + s));
+          }
+          if (ok) ptx::mma_commit(bar(kBarWEmpty + ws));
         }
-        if (ok) ptx::mma_commit(bar(kBarWEmpty + ws));
+        if (ok) ptx::mma_commit(bar(kBarAccFull + acc));
       }
-      if (ok) {
-        ptx::mma_commit(bar(kBarAcc));
-      } else {  // aborting: wait for the MMAs already issued
+      if (!ok) {  // aborting: wait for the MMAs already issued
         ptx::mma_commit(bar(kBarDrain));
         drain_bar(bar(kBarDrain), 0);
       }
     }
     __syncwarp();
-  } else {
-    // ---------------- dequantize, then epilogue ----------------
+  } else if (warp < kFirstEpiWarp) {
+    // ---------------- dequantize ----------------
     // Thread d = (row, half): row = d / 2 takes words 8 half .. 8 half + 7 of
     // its row, two 16-byte chunks read and stored in a rotated order (the
     // rotation also depends on the half) so that every 8-lane phase of the
@@ -245,64 +274,71 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rot = ((row >> 1) ^ hf) & 1;
     constexpr int kGPK = kKPerBlock / GS;
     bool ok = true;
-    for (int kb = 0; kb < KB; ++kb) {
-      const int qs = kb % kQStages;
-      if (!(ok = wait_bar(bar(kBarQFull + qs), (kb / kQStages) & 1, abort_flag, status))) break;
-      const uint8_t* qst = smem + L::kQOff + qs * kQStride;
-      const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64 + 32 * hf;
-      uint4 c[2];
+    int i = 0;  // k-blocks so far (Q and W stage uses)
+    for (int it = 0; it < ntiles && ok; ++it) {
+      for (int kb = 0; kb < KB; ++kb, ++i) {
+        const int qs = i % kQStages;
+        if (!(ok = wait_bar(bar(kBarQFull + qs), (i / kQStages) & 1, abort_flag, status))) break;
+        const uint8_t* qst = smem + L::kQOff + qs * kQStride;
+        const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64 + 32 * hf;
+        uint4 c[2];
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 1));
-      // fp16 bits of the scale and the zero point of this row, per group (rows
-      // past N read stale values: their outputs are never stored)
-      uint32_t s[kGPK], z[kGPK];
+        for (int jj = 0; jj < 2; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 1));
+        // fp16 bits of the scale and the zero point of this row, per group (rows
+        // past N read stale values: their outputs are never stored)
+        uint32_t s[kGPK], z[kGPK];
 #pragma unroll
-      for (int g = 0; g < kGPK; ++g) {
-        s[g] = reinterpret_cast<const uint16_t*>(qst + kQScaleOff + 256 * g)[row];
-        z[g] = (qst[kQZeroOff + 64 * g + (row >> 1)] >> (4 * (row & 1))) & 0xF;
-      }
-      ptx::mbar_arrive(bar(kBarQEmpty + qs));
-
-      const int ws = kb % kWStages;
-      if (!(ok = wait_bar(bar(kBarWEmpty + ws), ((kb / kWStages) & 1) ^ 1, abort_flag, status))) break;
-      __half2 s2[kGPK], zlo[kGPK], zhi[kGPK];
-#pragma unroll
-      for (int g = 0; g < kGPK; ++g) {
-        // fp16 bit patterns: s itself, 1024 + z = 0x6400 + z, -(64 + z) = 0xD400 + 16 z
-        s2[g] = u2h(s[g] * 0x00010001u);
-        zlo[g] = u2h((0x6400u + z[g]) * 0x00010001u);
-        zhi[g] = u2h((0xD400u + (z[g] << 4)) * 0x00010001u);
-      }
-      uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
-#pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        const int cj = 2 * hf + ((jj + rot) & 1);  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
-        const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
-#pragma unroll
-        for (int ww = 0; ww < 4; ++ww) {
-          // word 4 cj + ww holds inputs k0 .. k0 + 7 of group ww / (GS / 32)
-          // (word_k0 written out for this word: ww is a constant here)
-          constexpr int J = GS / 32;
-          const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
-          const int chunk = (k0 & 63) >> 3;  // 16-byte chunk (8 k) within the 64-k half
-          uint8_t* dst = wt + (k0 >> 6) * kWHalfBytes;
-          *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) = dequant_word(words[ww], zlo[g], zhi[g], s2[g]);
+        for (int g = 0; g < kGPK; ++g) {
+          s[g] = reinterpret_cast<const uint16_t*>(qst + kQScaleOff + 256 * g)[row];
+          z[g] = (qst[kQZeroOff + 64 * g + (row >> 1)] >> (4 * (row & 1))) & 0xF;
         }
+        ptx::mbar_arrive(bar(kBarQEmpty + qs));
+
+        const int ws = i % kWStages;
+        if (!(ok = wait_bar(bar(kBarWEmpty + ws), ((i / kWStages) & 1) ^ 1, abort_flag, status))) break;
+        __half2 s2[kGPK], zlo[kGPK], zhi[kGPK];
+#pragma unroll
+        for (int g = 0; g < kGPK; ++g) {
+          // fp16 bit patterns: s itself, 1024 + z = 0x6400 + z, -(64 + z) = 0xD400 + 16 z
+          s2[g] = u2h(s[g] * 0x00010001u);
+          zlo[g] = u2h((0x6400u + z[g]) * 0x00010001u);
+          zhi[g] = u2h((0xD400u + (z[g] << 4)) * 0x00010001u);
+        }
+        uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int cj = 2 * hf + ((jj + rot) & 1);  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
+          const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
+#pragma unroll
+          for (int ww = 0; ww < 4; ++ww) {
+            // word 4 cj + ww holds inputs k0 .. k0 + 7 of group ww / (GS / 32)
+            // (word_k0 written out for this word: ww is a constant here)
+            constexpr int J = GS / 32;
+            const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
+            const int chunk = (k0 & 63) >> 3;  // 16-byte chunk (8 k) within the 64-k half
+            uint8_t* dst = wt + (k0 >> 6) * kWHalfBytes;
+            *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) =
+                dequant_word(words[ww], zlo[g], zhi[g], s2[g]);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(bar(kBarWFull + ws));
       }
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(bar(kBarWFull + ws));
     }
-    if (ok && wait_bar(bar(kBarAcc), 0, abort_flag, status)) {
+  } else {
+    // ---------------- epilogue: accumulator -> fp16 y ----------------
+    const int quad = warp & 3;  // this warp may read TMEM lanes 32*quad .. +31
+    const int r = 32 * quad + lane;
+    for (int it = 0; it < ntiles; ++it) {
+      const int acc = it & 1;
+      if (!wait_bar(bar(kBarAccFull + acc), (it >> 1) & 1, abort_flag, status)) break;
       ptx::tc_fence_after();
-      const int quad = warp & 3;                     // this warp may read TMEM lanes 32*quad .. +31
-      const int colh = (warp - kFirstDeqWarp) >> 2;  // and takes half of the columns
-      const int r = 32 * quad + lane;
-      const int nn = n0 + r;
+      const int m0 = tile_m0(it), nn = tile_nt(it) * kBM + r;
 #pragma unroll 1
-      for (int c0 = colh * (BN / 2); c0 < (colh + 1) * (BN / 2); c0 += 32) {
+      for (int c0 = 0; c0 < BN; c0 += 32) {
         if (m0 + c0 >= M) break;
         uint32_t v[32];
-        ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)c0, v);
+        ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * BN + c0), v);
         ptx::tmem_wait_ld();
         if (nn < N) {
 #pragma unroll
@@ -315,6 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(kBarAccEmpty + acc));  // this thread's loads of the accumulator are done
     }
   }
 
@@ -322,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kWarpMma) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, BN);
+    ptx::tmem_dealloc(tmem_base, 2 * BN);
   }
 }
 
@@ -364,9 +402,10 @@ cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* sc
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
   }
-  dim3 grid((unsigned)((M + BN - 1) / BN), (unsigned)((N + kBM - 1) / kBM));
-  gemm_kernel<BN, GS><<<grid, kThreads, L::kAlloc, stream>>>(tx, qweight, scales, zeros, y, (int)M, (int)K, (int)N,
-                                                              status);
+  const int64_t tiles = ((M + BN - 1) / BN) * ((N + kBM - 1) / kBM);
+  const int ctas = (int)(tiles < device_info().sm_count ? tiles : device_info().sm_count);  // one per SM
+  gemm_kernel<BN, GS><<<ctas, kThreads, L::kAlloc, stream>>>(tx, qweight, scales, zeros, y, (int)M, (int)K, (int)N,
+                                                             status);
   return cudaGetLastError();
 }
 

@@ -771,7 +771,10 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
 // exit. Every contributor but the first starts its range inside the group, so
 // the group is its first one (slot 0); the first contributor holds the group
 // in slot 0 only if its range starts exactly at the group's first unit.
-__global__ void __launch_bounds__(128) gemv_fixup_kernel(const float* __restrict__ partial, __half* __restrict__ y,
+// (At most 32 registers a thread: 128 x 32 is what two resident GEMV CTAs
+// leave free on an SM, so fixup CTAs can be resident and waiting before the
+// GEMV's CTAs exit.)
+__global__ void __launch_bounds__(128, 16) gemv_fixup_kernel(const float* __restrict__ partial, __half* __restrict__ y,
                                                           int M, int K, int N, int KU, int P) {
   ptx::griddep_launch_dependents();
   const Range rg(K, N, KU, P);
@@ -788,12 +791,12 @@ __global__ void __launch_bounds__(128) gemv_fixup_kernel(const float* __restrict
   const int n = (int)(c_last - c_first);  // contributors after the first
   ptx::griddep_wait();
   float v = __ldcg(p + which_first * slot_floats);
-  for (int q0 = 1; q0 <= n; q0 += 8) {
-    float part[8];
+  for (int q0 = 1; q0 <= n; q0 += 4) {
+    float part[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) part[k] = q0 + k <= n ? __ldcg(p + (int64_t)(q0 + k) * cta_floats) : 0.f;
+    for (int k = 0; k < 4; ++k) part[k] = q0 + k <= n ? __ldcg(p + (int64_t)(q0 + k) * cta_floats) : 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v += part[k];
+    for (int k = 0; k < 4; ++k) v += part[k];
   }
   y[(int64_t)m * N + gi * kGroupBlocks * kRowsPerBlock + threadIdx.x] = __float2half_rn(v);
 }
