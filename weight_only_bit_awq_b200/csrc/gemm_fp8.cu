@@ -17,13 +17,14 @@
 // With the per-row power of two every nonzero |W8| lies in [448/30, 448]: all
 // E4M3 normal numbers, so each weight keeps 4 significant bits.
 //
-// The GEMM has the structure of the fp16 one (gemm_tc.cu): one 128-channel x
-// BN-token tile per CTA, warp 0 loads x8 by TMA (one 128-byte-wide box per
-// 128-input k-block, 128-byte swizzle), warp 1 issues 4 MMAs of K = 32 per
-// k-block, warp 2 copies the packed codes and the tile's scale and zero rows,
-// warps 3-10 dequantize (two threads per weight row, half of its codes each:
-// two warps per SM sub-partition hide the conversion latency) and then run the
-// epilogue (warps w and w + 4 share TMEM lanes and split the columns). Every
+// The GEMM has the structure of the fp16 one (gemm_tc.cu): persistent, one
+// CTA per SM over 128-channel x BN-token tiles with two tensor-memory
+// accumulators; warp 0 loads x8 by TMA (one 128-byte-wide box per 128-input
+// k-block, 128-byte swizzle), warp 1 issues 4 MMAs of K = 32 per k-block,
+// warp 2 copies the packed codes and the tile's scale and zero rows, warps
+// 3-10 dequantize (two threads per weight row, half of its codes each: two
+// warps per SM sub-partition hide the conversion latency) and warps 11-14 run
+// the epilogue of one tile while the next is accumulated. Every
 // mbarrier wait is bounded; on expiry AWQ_ERR_TIMEOUT goes to the status word
 // and the CTA drains and exits.
 #include <cuda_fp8.h>
@@ -200,13 +201,14 @@ constexpr int kQScaleOff = kQBytes, kQZeroOff = kQScaleOff + 4 * 256;
 constexpr int kQStride = kQZeroOff + 4 * 64;
 constexpr int kWBytes = kBM * kKPerBlock;  // 16 KiB: 128 rows x 128 E4M3 weights
 constexpr int kWarpX = 0, kWarpMma = 1, kWarpQ = 2, kFirstDeqWarp = 3, kNumDeqWarps = 8;
-constexpr int kDeqThreads = kNumDeqWarps * 32;
-constexpr int kThreads = (kFirstDeqWarp + kNumDeqWarps) * 32;
+constexpr int kFirstEpiWarp = kFirstDeqWarp + kNumDeqWarps, kNumEpiWarps = 4;
+constexpr int kDeqThreads = kNumDeqWarps * 32, kEpiThreads = kNumEpiWarps * 32;
+constexpr int kThreads = (kFirstEpiWarp + kNumEpiWarps) * 32;
 
 constexpr int kBarXFull = 0, kBarXEmpty = kBarXFull + kXStages, kBarWFull = kBarXEmpty + kXStages,
               kBarWEmpty = kBarWFull + kWStages, kBarQFull = kBarWEmpty + kWStages,
-              kBarQEmpty = kBarQFull + kQStages, kBarAcc = kBarQEmpty + kQStages, kBarDrain = kBarAcc + 1,
-              kNumBars = kBarDrain + 1;
+              kBarQEmpty = kBarQFull + kQStages, kBarAccFull = kBarQEmpty + kQStages, kBarAccEmpty = kBarAccFull + 2,
+              kBarDrain = kBarAccEmpty + 2, kNumBars = kBarDrain + 1;
 
 template <int BN>
 struct Layout {
@@ -224,6 +226,10 @@ static_assert(Layout<256>::kAlloc <= 232448, "shared memory budget");
 using ptx::drain_bar;
 using ptx::wait_bar;
 
+// Persistent: CTA c computes tiles c, c + P, ... (P = gridDim.x; tile t is
+// token tile t % MT of channel tile t / MT); the rings run on across tiles and
+// the two accumulators let the epilogue warps drain one tile while the MMA
+// warp fills the next.
 template <int BN, int GS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict__ sx,
@@ -239,9 +245,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BN;
-  const int n0 = blockIdx.y * kBM;
   const int KB = K / kKPerBlock;
+  const int MT = (M + BN - 1) / BN, NT = (N + kBM - 1) / kBM, T = MT * NT;
+  const int P = gridDim.x;
+  const int ntiles = blockIdx.x < T ? (T - 1 - (int)blockIdx.x) / P + 1 : 0;  // tiles of this CTA
+  auto tile_m0 = [&](int it) { return ((int)blockIdx.x + it * P) % MT * BN; };
+  auto tile_nt = [&](int it) { return ((int)blockIdx.x + it * P) / MT; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kXStages; ++i) {
@@ -256,14 +265,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(bar(kBarQFull + i), 33);  // the codes' byte count + 32 cp.async arrivals
       ptx::mbar_init(bar(kBarQEmpty + i), kDeqThreads);
     }
-    ptx::mbar_init(bar(kBarAcc), 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(kBarAccFull + i), 1);
+      ptx::mbar_init(bar(kBarAccEmpty + i), kEpiThreads);
+    }
     ptx::mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
   }
   if (warp == kWarpX && lane == 0) ptx::prefetch_tensormap(&tmap_x);
   if (warp == kWarpMma) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), BN);
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 2 * BN);
     ptx::tmem_relinquish();
     ptx::tc_fence_before();
   }
@@ -274,49 +286,57 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpX) {
     // ---------------- x8 producer: one 128-byte-wide box per k-block ----------------
     if (lane == 0) {
-      int kb = 0;
-      for (; kb < KB; ++kb) {
-        const int s = kb % kXStages;
-        if (!wait_bar(bar(kBarXEmpty + s), ((kb / kXStages) & 1) ^ 1, abort_flag, status)) break;
-        ptx::mbar_arrive_expect_tx(bar(kBarXFull + s), L::kXBytes);
-        ptx::tma_load_2d(sbase + L::kXOff + s * L::kXBytes, &tmap_x, kb * kKPerBlock, m0, bar(kBarXFull + s));
+      int i = 0;
+      bool ok = true;
+      for (int it = 0; it < ntiles && ok; ++it) {
+        const int m0 = tile_m0(it);
+        for (int kb = 0; kb < KB; ++kb, ++i) {
+          const int s = i % kXStages;
+          if (!(ok = wait_bar(bar(kBarXEmpty + s), ((i / kXStages) & 1) ^ 1, abort_flag, status))) break;
+          ptx::mbar_arrive_expect_tx(bar(kBarXFull + s), L::kXBytes);
+          ptx::tma_load_2d(sbase + L::kXOff + s * L::kXBytes, &tmap_x, kb * kKPerBlock, m0, bar(kBarXFull + s));
+        }
       }
-      if (kb < KB)  // aborting: let the copies already issued land
-        for (int j = (kb > kXStages ? kb - kXStages : 0); j < kb; ++j)
+      if (!ok)  // aborting: let the copies already issued land
+        for (int j = (i > kXStages ? i - kXStages : 0); j < i; ++j)
           drain_bar(bar(kBarXFull + j % kXStages), (j / kXStages) & 1);
     }
     __syncwarp();
   } else if (warp == kWarpQ) {
     // ---------------- packed-weight producer (as in the fp16 GEMM) ----------------
     constexpr int kGPK = kKPerBlock / GS;
-    const int64_t NB = N / kRowsPerBlock, gi = blockIdx.y;
-    const uint32_t qbytes = (uint32_t)(group_rows(gi, NB) * 1024);
-    int kb = 0;
-    for (; kb < KB; ++kb) {
-      const int s = kb % kQStages;
-      bool ok = true;
-      if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((kb / kQStages) & 1) ^ 1, abort_flag, status);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const uint32_t st = sbase + L::kQOff + s * kQStride;
-      if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qbytes);
-      __syncwarp();
-      if (lane == 0)
-        ptx::bulk_g2s(st, qweight + unit_first_block(gi, kb, KB, NB) * kWordsPerBlock, qbytes, bar(kBarQFull + s));
-      for (int p = lane; p < kGPK * 16; p += 32) {  // kGPK rows of 128 scales: 16 B = 8 output channels
-        const int g = p >> 4, l = p & 15;
-        if (n0 + 8 * l < N)
-          ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
+    const int64_t NB = N / kRowsPerBlock;
+    int i = 0;
+    bool ok = true;
+    for (int it = 0; it < ntiles && ok; ++it) {
+      const int64_t gi = tile_nt(it);
+      const int n0 = (int)gi * kBM;
+      const uint32_t qbytes = (uint32_t)(group_rows(gi, NB) * 1024);
+      for (int kb = 0; kb < KB; ++kb, ++i) {
+        const int s = i % kQStages;
+        if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((i / kQStages) & 1) ^ 1, abort_flag, status);
+        if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+        const uint32_t st = sbase + L::kQOff + s * kQStride;
+        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qbytes);
+        __syncwarp();
+        if (lane == 0)
+          ptx::bulk_g2s(st, qweight + unit_first_block(gi, kb, KB, NB) * kWordsPerBlock, qbytes, bar(kBarQFull + s));
+        for (int p = lane; p < kGPK * 16; p += 32) {  // kGPK rows of 128 scales: 16 B = 8 output channels
+          const int g = p >> 4, l = p & 15;
+          if (n0 + 8 * l < N)
+            ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
+        }
+        for (int p = lane; p < kGPK * 8; p += 32) {  // kGPK rows of 64 zero bytes: 8 B = 16 output channels
+          const int g = p >> 3, l = p & 7;
+          if (n0 + 16 * l < N)
+            ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l,
+                            zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
+        }
+        ptx::cp_async_arrive_noinc(bar(kBarQFull + s));
       }
-      for (int p = lane; p < kGPK * 8; p += 32) {  // kGPK rows of 64 zero bytes: 8 B = 16 output channels
-        const int g = p >> 3, l = p & 7;
-        if (n0 + 16 * l < N)
-          ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l,
-                          zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
-      }
-      ptx::cp_async_arrive_noinc(bar(kBarQFull + s));
     }
-    if (kb < KB && lane == 0)
-      for (int j = (kb > kQStages ? kb - kQStages : 0); j < kb; ++j)
+    if (!ok && lane == 0)
+      for (int j = (i > kQStages ? i - kQStages : 0); j < i; ++j)
         drain_bar(bar(kBarQFull + j % kQStages), (j / kQStages) & 1);
     __syncwarp();
   } else if (warp == kWarpMma) {
@@ -324,30 +344,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = ptx::idesc_e4m3_f32(kBM, BN);
       bool ok = true;
-      for (int kb = 0; kb < KB && ok; ++kb) {
-        const int ws = kb % kWStages, xs = kb % kXStages;
-        if (!(ok = wait_bar(bar(kBarWFull + ws), (kb / kWStages) & 1, abort_flag, status))) break;
-        if (!(ok = wait_bar(bar(kBarXFull + xs), (kb / kXStages) & 1, abort_flag, status))) break;
+      int i = 0;  // k-blocks so far (W and x stage uses)
+      for (int it = 0; it < ntiles && ok; ++it) {
+        const int acc = it & 1;
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        if (!(ok = wait_bar(bar(kBarAccEmpty + acc), ((it >> 1) & 1) ^ 1, abort_flag, status))) break;
         ptx::tc_fence_after();
-        const uint32_t a_base = sbase + L::kWOff + ws * kWBytes;
-        const uint32_t b_base = sbase + L::kXOff + xs * L::kXBytes;
+        for (int kb = 0; kb < KB; ++kb, ++i) {
+          const int ws = i % kWStages, xs = i % kXStages;
+          if (!(ok = wait_bar(bar(kBarWFull + ws), (i / kWStages) & 1, abort_flag, status))) break;
+          if (!(ok = wait_bar(bar(kBarXFull + xs), (i / kXStages) & 1, abort_flag, status))) break;
+          ptx::tc_fence_after();
+          const uint32_t a_base = sbase + L::kWOff + ws * kWBytes;
+          const uint32_t b_base = sbase + L::kXOff + xs * L::kXBytes;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_f8f6f4_ss(tmem_base, ptx::desc_kmajor_sw128(a_base + 32 * kk),
-                             ptx::desc_kmajor_sw128(b_base + 32 * kk), idesc, (kb | kk) != 0);
-        ptx::mma_commit(bar(kBarXEmpty + xs));
-        ptx::mma_commit(bar(kBarWEmpty + ws));
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_f8f6f4_ss(d_tmem, ptx::desc_kmajor_sw128(a_base + 32 * kk),
+                               ptx::desc_kmajor_sw128(b_base + 32 * kk), idesc, (kb | kk) != 0);
+          ptx::mma_commit(bar(kBarXEmpty + xs));
+          ptx::mma_commit(bar(kBarWEmpty + ws));
+        }
+        if (ok) ptx::mma_commit(bar(kBarAccFull + acc));
       }
-      if (ok) {
-        ptx::mma_commit(bar(kBarAcc));
-      } else {  // aborting: wait for the MMAs already issued
+      if (!ok) {  // aborting: wait for the MMAs already issued
         ptx::mma_commit(bar(kBarDrain));
         drain_bar(bar(kBarDrain), 0);
       }
     }
     __syncwarp();
-  } else {
-    // ---------------- dequantize to E4M3, then epilogue ----------------
+  } else if (warp < kFirstEpiWarp) {
+    // ---------------- dequantize to E4M3 ----------------
     // Thread d = (row, half): row = d / 2 takes codes words 8 half .. 8 half + 7
     // of its row (two 16-byte chunks, read in a rotated order so that the
     // warp's shared loads are bank-conflict free).
@@ -355,63 +381,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = d >> 1, hf = d & 1;
     const int rot = (row >> 1) & 1;
     constexpr int kGPK = kKPerBlock / GS;
-    const int nn = n0 + row;
-    const int e = nn < N ? row_exp[nn] : 0;
-    const float pow2e = pow2f(e);
     bool ok = true;
-    for (int kb = 0; kb < KB; ++kb) {
-      const int qs = kb % kQStages;
-      if (!(ok = wait_bar(bar(kBarQFull + qs), (kb / kQStages) & 1, abort_flag, status))) break;
-      const uint8_t* qst = smem + L::kQOff + qs * kQStride;
-      const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64 + 32 * hf;
-      uint4 c[2];
+    int i = 0;  // k-blocks so far (Q and W stage uses)
+    for (int it = 0; it < ntiles && ok; ++it) {
+      const int nn = tile_nt(it) * kBM + row;
+      const float pow2e = pow2f(nn < N ? row_exp[nn] : 0);
+      for (int kb = 0; kb < KB; ++kb, ++i) {
+        const int qs = i % kQStages;
+        if (!(ok = wait_bar(bar(kBarQFull + qs), (i / kQStages) & 1, abort_flag, status))) break;
+        const uint8_t* qst = smem + L::kQOff + qs * kQStride;
+        const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64 + 32 * hf;
+        uint4 c[2];
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 1));
-      // scale and zero point of this row, per group (rows past N read stale
-      // values: their outputs are never stored)
-      uint32_t sb[kGPK], z[kGPK];
+        for (int jj = 0; jj < 2; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 1));
+        // scale and zero point of this row, per group (rows past N read stale
+        // values: their outputs are never stored)
+        uint32_t sb[kGPK], z[kGPK];
 #pragma unroll
-      for (int g = 0; g < kGPK; ++g) {
-        sb[g] = reinterpret_cast<const uint16_t*>(qst + kQScaleOff + 256 * g)[row];
-        z[g] = (qst[kQZeroOff + 64 * g + (row >> 1)] >> (4 * (row & 1))) & 0xF;
-      }
-      ptx::mbar_arrive(bar(kBarQEmpty + qs));
-
-      const int ws = kb % kWStages;
-      if (!(ok = wait_bar(bar(kBarWEmpty + ws), ((kb / kWStages) & 1) ^ 1, abort_flag, status))) break;
-      GroupConsts gc[kGPK];
-#pragma unroll
-      for (int g = 0; g < kGPK; ++g) gc[g] = group_consts(sb[g], z[g], pow2e);
-      uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
-#pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        const int cj = 2 * hf + ((jj + rot) & 1);  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
-        const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
-#pragma unroll
-        for (int ww = 0; ww < 4; ++ww) {
-          // word 4 cj + ww holds inputs k0 .. k0 + 7 of group ww / (GS / 32)
-          constexpr int J = GS / 32;
-          const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
-          const int chunk = k0 >> 4;  // 16-byte chunk (16 inputs) of the 128-byte row
-          *reinterpret_cast<uint2*>(wt + ((chunk ^ (row & 7)) << 4) + (k0 & 8)) =
-              w8_word(words[ww], gc[g].zlo, gc[g].zhi, gc[g].s2);
+        for (int g = 0; g < kGPK; ++g) {
+          sb[g] = reinterpret_cast<const uint16_t*>(qst + kQScaleOff + 256 * g)[row];
+          z[g] = (qst[kQZeroOff + 64 * g + (row >> 1)] >> (4 * (row & 1))) & 0xF;
         }
+        ptx::mbar_arrive(bar(kBarQEmpty + qs));
+
+        const int ws = i % kWStages;
+        if (!(ok = wait_bar(bar(kBarWEmpty + ws), ((i / kWStages) & 1) ^ 1, abort_flag, status))) break;
+        GroupConsts gc[kGPK];
+#pragma unroll
+        for (int g = 0; g < kGPK; ++g) gc[g] = group_consts(sb[g], z[g], pow2e);
+        uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int cj = 2 * hf + ((jj + rot) & 1);  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
+          const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
+#pragma unroll
+          for (int ww = 0; ww < 4; ++ww) {
+            // word 4 cj + ww holds inputs k0 .. k0 + 7 of group ww / (GS / 32)
+            constexpr int J = GS / 32;
+            const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
+            const int chunk = k0 >> 4;  // 16-byte chunk (16 inputs) of the 128-byte row
+            *reinterpret_cast<uint2*>(wt + ((chunk ^ (row & 7)) << 4) + (k0 & 8)) =
+                w8_word(words[ww], gc[g].zlo, gc[g].zhi, gc[g].s2);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(bar(kBarWFull + ws));
       }
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(bar(kBarWFull + ws));
     }
-    if (ok && wait_bar(bar(kBarAcc), 0, abort_flag, status)) {
+  } else {
+    // ---------------- epilogue: y = fp16(acc * sx[m] * 2^-e[n]) ----------------
+    const int quad = warp & 3;  // this warp may read TMEM lanes 32*quad .. +31
+    const int r = 32 * quad + lane;
+    for (int it = 0; it < ntiles; ++it) {
+      const int acc = it & 1;
+      if (!wait_bar(bar(kBarAccFull + acc), (it >> 1) & 1, abort_flag, status)) break;
       ptx::tc_fence_after();
-      const int quad = warp & 3;                          // this warp may read TMEM lanes 32*quad .. +31
-      const int colh = (warp - kFirstDeqWarp) >> 2;       // and takes half of the columns
-      const int r = 32 * quad + lane;
-      const int n = n0 + r;
+      const int m0 = tile_m0(it), n = tile_nt(it) * kBM + r;
       const float pow2ne = pow2f(-(n < N ? row_exp[n] : 0));
 #pragma unroll 1
-      for (int c0 = colh * (BN / 2); c0 < (colh + 1) * (BN / 2); c0 += 32) {
+      for (int c0 = 0; c0 < BN; c0 += 32) {
         if (m0 + c0 >= M) break;
         uint32_t v[32];
-        ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)c0, v);
+        ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * BN + c0), v);
         ptx::tmem_wait_ld();
         if (n < N) {
 #pragma unroll
@@ -427,6 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(kBarAccEmpty + acc));  // this thread's loads of the accumulator are done
     }
   }
 
@@ -434,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kWarpMma) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, BN);
+    ptx::tmem_dealloc(tmem_base, 2 * BN);
   }
 }
 
@@ -478,8 +511,9 @@ cudaError_t launch_bn(const uint8_t* x8, const float* sx, const uint32_t* qweigh
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
   }
-  dim3 grid((unsigned)((M + BN - 1) / BN), (unsigned)((N + kBM - 1) / kBM));
-  gemm_fp8_kernel<BN, GS><<<grid, kThreads, L::kAlloc, stream>>>(tx, sx, qweight, scales, zeros, row_exp, y, (int)M,
+  const int64_t tiles = ((M + BN - 1) / BN) * ((N + kBM - 1) / kBM);
+  const int ctas = (int)(tiles < device_info().sm_count ? tiles : device_info().sm_count);  // one per SM
+  gemm_fp8_kernel<BN, GS><<<ctas, kThreads, L::kAlloc, stream>>>(tx, sx, qweight, scales, zeros, row_exp, y, (int)M,
                                                                   (int)K, (int)N, status);
   return cudaGetLastError();
 }
