@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict__ sx,
                     const uint32_t* __restrict__ qweight, const __half* __restrict__ scales,
                     const uint8_t* __restrict__ zeros, const int8_t* __restrict__ row_exp, __half* __restrict__ y,
-                    int M, int K, int N, uint32_t* status) {
+                    int M, int K, int N, int GM, uint32_t* status) {
   using L = Layout<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -249,8 +249,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int MT = (M + BN - 1) / BN, NT = (N + kBM - 1) / kBM, T = MT * NT;
   const int P = gridDim.x;
   const int ntiles = blockIdx.x < T ? (T - 1 - (int)blockIdx.x) / P + 1 : 0;  // tiles of this CTA
-  auto tile_m0 = [&](int it) { return ((int)blockIdx.x + it * P) % MT * BN; };
-  auto tile_nt = [&](int it) { return ((int)blockIdx.x + it * P) / MT; };
+  // Tile order: blocks of GM token tiles; within a block, token tile fastest,
+  // then channel tile. The x of one block stays in L2 while the block's
+  // channel tiles stream past it.
+  auto tile_mn = [&](int it, int& mt, int& nt) {
+    const int t = (int)blockIdx.x + it * P;
+    const int blk = t / (GM * NT), w = t - blk * GM * NT;
+    const int gb = min(GM, MT - blk * GM);  // token tiles in this block
+    mt = blk * GM + w % gb;
+    nt = w / gb;
+  };
+  auto tile_m0 = [&](int it) {
+    int mt, nt;
+    tile_mn(it, mt, nt);
+    return mt * BN;
+  };
+  auto tile_nt = [&](int it) {
+    int mt, nt;
+    tile_mn(it, mt, nt);
+    return nt;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kXStages; ++i) {
@@ -471,6 +489,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Token tiles per block of the tile order: as many as keep the block's x
+// (tiles x BN tokens x K inputs) within ~48 MB of the 126 MB L2, at least one.
+int token_tiles_per_block(int64_t M, int64_t K, int BN, int xbytes) {
+  const int64_t mt = (M + BN - 1) / BN;
+  int64_t g = (int64_t(48) << 20) / ((int64_t)BN * K * xbytes);
+  if (g < 1) g = 1;
+  return (int)(g < mt ? g : mt);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -514,7 +541,8 @@ cudaError_t launch_bn(const uint8_t* x8, const float* sx, const uint32_t* qweigh
   const int64_t tiles = ((M + BN - 1) / BN) * ((N + kBM - 1) / kBM);
   const int ctas = (int)(tiles < device_info().sm_count ? tiles : device_info().sm_count);  // one per SM
   gemm_fp8_kernel<BN, GS><<<ctas, kThreads, L::kAlloc, stream>>>(tx, sx, qweight, scales, zeros, row_exp, y, (int)M,
-                                                                  (int)K, (int)N, status);
+                                                                  (int)K, (int)N,
+                                                                  token_tiles_per_block(M, K, BN, 1), status);
   return cudaGetLastError();
 }
 
@@ -522,7 +550,11 @@ template <int GS>
 cudaError_t launch_gs(const uint8_t* x8, const float* sx, const uint32_t* qweight, const __half* scales,
                       const uint8_t* zeros, const int8_t* row_exp, __half* y, int64_t M, int64_t K, int64_t N,
                       uint32_t* status, cudaStream_t stream) {
-  if (M > 128) return launch_bn<256, GS>(x8, sx, qweight, scales, zeros, row_exp, y, M, K, N, status, stream);
+  // 256-token tiles unless they cannot give every SM a tile and 128-token
+  // tiles would give it more (e.g. K=14336, N=4096, M=512: 64 against 128 tiles)
+  const int64_t nt = (N + kBM - 1) / kBM;
+  if (M > 128 && ((M + 255) / 256 * nt >= device_info().sm_count || (M + 127) / 128 * nt <= (M + 255) / 256 * nt))
+    return launch_bn<256, GS>(x8, sx, qweight, scales, zeros, row_exp, y, M, K, N, status, stream);
   return launch_bn<128, GS>(x8, sx, qweight, scales, zeros, row_exp, y, M, K, N, status, stream);
 }
 
