@@ -403,11 +403,13 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       int jj = (int)(u0 % rg.UPG), s = 0, ph = 0;
       for (int i = 0; i < n_units; ++i) {
         if (!ptx::wait_bar(xland(s), ph, abort_flag, status)) break;
-        const int64_t kb0 = (int64_t)jj * KU;
-        const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
         const uint8_t* st = smem + s * L.bytes;
-        for (int j = 0; j < ku; ++j) {
-          float lo = 0.f, hi = 0.f;
+        // All KU k-blocks of the stage at once (their latency chains overlap);
+        // slots past a short last unit get values that are never read.
+        float lo[KU], hi[KU];
+#pragma unroll
+        for (int j = 0; j < KU; ++j) {
+          lo[j] = hi[j] = 0.f;
           if (m < M) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -415,20 +417,25 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
                                                               64 * t4 + 16 * q);
               const float2 p0 = __half22float2(u32_as_h2(v.x)), p1 = __half22float2(u32_as_h2(v.y));
               const float2 p2 = __half22float2(u32_as_h2(v.z)), p3 = __half22float2(u32_as_h2(v.w));
-              lo += (p0.x + p0.y) + (p2.x + p2.y);
-              hi += (p1.x + p1.y) + (p3.x + p3.y);
+              lo[j] += (p0.x + p0.y) + (p2.x + p2.y);
+              hi[j] += (p1.x + p1.y) + (p3.x + p3.y);
             }
           }
+        }
 #pragma unroll
-          for (int off = 1; off < GS / 32; off <<= 1) {
-            lo += __shfl_xor_sync(0xffffffffu, lo, off);
-            hi += __shfl_xor_sync(0xffffffffu, hi, off);
+        for (int off = 1; off < GS / 32; off <<= 1)
+#pragma unroll
+          for (int j = 0; j < KU; ++j) {
+            lo[j] += __shfl_xor_sync(0xffffffffu, lo[j], off);
+            hi[j] += __shfl_xor_sync(0xffffffffu, hi[j], off);
           }
-          if (t4 % (GS / 32) == 0 && m < M) {
-            const int gk = t4 / (GS / 32);
+        if (t4 % (GS / 32) == 0 && m < M) {
+          const int gk = t4 / (GS / 32);
+#pragma unroll
+          for (int j = 0; j < KU; ++j) {
             float* xs = reinterpret_cast<float*>(smem + s * L.bytes + L.xs + (j * kGPK + gk) * kKbXsBytes);
-            xs[2 * m] = 1024.f * lo + 64.f * hi;
-            xs[2 * m + 1] = lo + hi;
+            xs[2 * m] = 1024.f * lo[j] + 64.f * hi[j];
+            xs[2 * m + 1] = lo[j] + hi[j];
           }
         }
         __syncwarp();
