@@ -32,8 +32,12 @@
 //     shared memory). The MMA sums over k, so any permutation of k applied to
 //     A and B alike is allowed: a lane pairs the k it loaded with the fragment
 //     slots it owns. The fp32 result of a k-block is sum_k x (q - z) over one
-//     group; y += s * that, in fp32, so no weight is rounded.
-//   warp 9 (M <= 8 only): per-k-block sums of x, see block_mma_lohi.
+//     group; y += s * that, in fp32, so no weight is rounded. For M <= 2 with
+//     groups of 128 the consumers use integer MMAs instead (mma.sync
+//     m16n8k32, u8 codes x s8 digits of x; see the integer path below).
+//   warp 9 (M <= 8 only) reads each stage's x first: per-k-block sums of x for
+//     the lo/hi path (see block_mma_lohi), or, on the integer path, the
+//     block fixed-point digits and coefficients of x.
 //
 // Output. A warp that saw all k-blocks of its row block writes fp16 y. A row
 // block split between CTAs (only the first and the last group of a CTA's
