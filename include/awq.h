@@ -143,7 +143,11 @@ awq_status awq_w4a16_gemv(const void* x, const void* qweight, const void* scales
 /* Context-stage (prefill) W4A16 GEMM for any M (README "New Optimization of
  * Context Stage": the prompt is processed as one batch of tokens): same
  * result as awq_w4a16_gemv, on the tcgen05 tensor cores with fp32
- * accumulation in tensor memory. */
+ * accumulation in tensor memory. For M > AWQ_GEMV_MAX_M, where whole output
+ * tiles would leave the last wave of SMs short, the k-range of the last tiles
+ * is split between CTAs ("stream-K") and a second kernel adds the fp32 parts,
+ * which live in the workspace, in a fixed order: results are deterministic
+ * for a given device (SM count). */
 awq_status awq_w4a16_gemm(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
                           int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,
                           void* stream);
@@ -226,8 +230,8 @@ awq_status awq_w4a16_gemv_no_alloc(const void* x, const void* qweight, const voi
                                    void* y, int64_t M, int64_t K, int64_t N, int group, void* stream);
 
 /* Number of kernels awq_linear launches for these sizes on the current device
- * (1, or 2 when the decode GEMV also runs its split-row fixup kernel; 0 for
- * M == 0 or invalid sizes). Host only. For launch accounting and graph planning;
+ * (1, or 2 when the decode GEMV runs its split-row fixup kernel or the GEMM
+ * its stream-K fixup kernel; 0 for M == 0 or invalid sizes). Host only. For launch accounting and graph planning;
  * the pages have no counterpart. */
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group);
 

@@ -73,6 +73,23 @@ def test_workspace_bytes():
     assert awq.awq_workspace_bytes(32, 4096, 4096) >= awq.awq_workspace_bytes(1, 4096, 4096)
 
 
+def test_gemm_schedule_on_148_sms():
+    # Without a device the library plans for 148 SMs. Tiles are 128 channels x
+    # 256 tokens here. Stream-K (a second, fixup kernel, and two fp32 slots of
+    # 128 x 256 per SM in the workspace) when whole tiles fill under 80 % of the
+    # SM-tile slots: 448 tiles = 3.03 waves at M = 512 (76 %), but not 1792 =
+    # 12.1 waves at M = 2048 (93 %) or 7168 = 48.4 at M = 8192.
+    slots = 256 + 148 * 2 * 256 * 128 * 4
+    for M, launches in ((512, 2), (2048, 1), (8192, 1)):
+        assert awq.awq_linear_launches(M, 4096, 28672, 128) == launches
+        assert (awq.awq_workspace_bytes(M, 4096, 28672) >= slots) == (launches == 2)
+    # never for decode sizes: those workspaces stay what the GEMV needs
+    assert awq.awq_linear_launches(32, 14336, 4096, 128) in (1, 2)
+    assert awq.awq_workspace_bytes(32, 14336, 4096) < slots
+    # at least 8 k-blocks per SM: K = 128 with 8 tiles stays data-parallel
+    assert awq.awq_linear_launches(40, 128, 1024, 128) == 1
+
+
 def _linear(fn, x=FAKE, q=FAKE2, s=FAKE3, z=FAKE4, y=FAKE5, M=1, K=4096, N=4096, group=128, ws=FAKE6,
             ws_bytes=1 << 30):
     return getattr(L, fn)(x, q, s, z, y, M, K, N, group, ws, ws_bytes, None)
@@ -128,7 +145,8 @@ def test_valid_arguments_without_a_device_stop_at_the_device_check():
 def test_linear_launch_counts():
     assert awq.awq_linear_launches(0, 4096, 4096) == 0
     assert awq.awq_linear_launches(1, 4000, 4096) == 0
-    assert awq.awq_linear_launches(2048, 4096, 4096) == 1          # the GEMM: one kernel
+    assert awq.awq_linear_launches(8192, 4096, 4096) == 1          # the GEMM, data-parallel: one kernel
+    assert awq.awq_linear_launches(300, 1024, 9600) == 2           # stream-K: the GEMM and its fixup
     assert awq.awq_linear_launches(1, 4096, 4096) in (1, 2)        # the GEMV, plus its fixup when rows are split
 
 

@@ -119,6 +119,55 @@ def test_gemv_and_gemm_agree_closely():
     check_close(y2, y_ref, b)
 
 
+# ---- prefill GEMM with the stream-K schedule --------------------------------
+# When whole 128-channel x BN-token tiles would leave the last wave of SMs
+# short, the k-blocks of the last tiles are split evenly between the CTAs and
+# a fixup kernel adds the fp32 parts in CTA order. Shapes (M, K, N, group):
+# every tile split many ways (8 tiles on all SMs); whole data-parallel tiles
+# followed by split ones; 256-token tiles with a ragged last token tile
+# (M = 300, 513); groups of 64 and 32.
+STREAM_K_CASES = [(40, 24576, 1024, 128), (40, 1024, 38400, 128), (300, 1024, 9600, 128), (513, 2048, 6400, 128),
+                  (40, 2048, 19200, 64), (40, 2048, 19200, 32)]
+
+
+@pytest.mark.parametrize("M,K,N,group", STREAM_K_CASES)
+def test_gemm_stream_k_matches_oracle(M, K, N, group):
+    assert awq.awq_linear_launches(M, K, N, group) == 2  # the schedule is stream-K here
+    W, dev, hp = _packed(N, K, f"sk{K}x{N}", group=group)
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"sk{K}x{N}/x{M}"), M, K, 1.0)
+    xd = to_dev(x.view(np.uint16), torch.float16)
+    ws = awq.new_workspace(M, K, N, xd.device, group)
+    ys = [host(awq.awq_w4a16_gemm(xd, *dev, N, ws, group), np.float16) for _ in range(2)]
+    st = awq.awq_get_status(ws)
+    assert st == awq.AWQ_OK, awq.awq_status_string(st)
+    assert (ys[0].view(np.uint16) == ys[1].view(np.uint16)).all()  # deterministic
+    # all tokens on rows of every 128-channel tile (its first and last row and
+    # random ones), about 8e7 oracle multiply-adds
+    rng = np.random.default_rng(M + N)
+    per_tile = max(2, int(8e7 / (M * K * ((N + 127) // 128))))
+    rows = set()
+    for n0 in range(0, N, 128):
+        hi = min(N, n0 + 128)
+        rows |= {n0, hi - 1} | set(rng.integers(n0, hi, per_tile - 2).tolist())
+    rows = np.array(sorted(rows), dtype=np.int64)
+    y_ref, b = oracle_rows(x, *hp, N, K, rows, group)
+    check_close(ys[0][:, rows], y_ref, b, f"stream-K gemm M={M} K={K} N={N} g={group}")
+
+
+def test_gemm_stream_k_one_hot_gives_the_dequantized_weight_exactly():
+    # one nonzero input per token: each output is one dequantized weight, and
+    # the fp32 parts of the split tiles (all but one exactly zero) add up to it
+    M, K, N = 40, 24576, 1024
+    W, dev, hp = _packed(N, K, "sk_onehot")
+    q, z, s = oracle.unpack(*hp, N, K)
+    wh = oracle.dequant(q, z, s)
+    ks = np.random.default_rng(7).integers(0, K, M)
+    x = np.zeros((M, K), np.float16)
+    x[np.arange(M), ks] = 1.0
+    y = _run(awq.awq_w4a16_gemm, x, dev, N)
+    assert (y.view(np.uint16) == wh[:, ks].T.view(np.uint16)).all()
+
+
 # ---- full-size workloads, sampled against the oracle ----------------------
 
 DECODE_CASES = [("single_4096", "linear", 1)]

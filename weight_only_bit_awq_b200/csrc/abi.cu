@@ -129,9 +129,10 @@ awq_status gemv_impl(const LinearArgs& a, cudaStream_t stream) {
 }
 
 awq_status gemm_impl(const LinearArgs& a, cudaStream_t stream) {
+  const GemmPlan p = plan_gemm(a.M, a.K, a.N, device_info().sm_count);
   cudaError_t e = launch_gemm(static_cast<const __half*>(a.x), static_cast<const uint32_t*>(a.qweight),
                               static_cast<const __half*>(a.scales), static_cast<const uint8_t*>(a.zeros),
-                              static_cast<__half*>(a.y), a.M, a.K, a.N, a.group, status_word(a.workspace), stream);
+                              static_cast<__half*>(a.y), a.M, a.K, a.N, a.group, p, a.workspace, stream);
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
@@ -156,6 +157,9 @@ size_t awq_workspace_bytes(int64_t M, int64_t K, int64_t N, int group) {
   size_t need = kWsHeaderBytes;
   if (M >= 1 && M <= AWQ_GEMV_MAX_M) {
     const GemvPlan p = plan_gemv(M, K, N, group, sm_count_or_default());
+    if (p.ws_bytes > need) need = p.ws_bytes;
+  } else if (M > AWQ_GEMV_MAX_M) {
+    const GemmPlan p = plan_gemm(M, K, N, sm_count_or_default());
     if (p.ws_bytes > need) need = p.ws_bytes;
   }
   return need;
@@ -317,7 +321,7 @@ awq_status awq_w4a8_gemm(const void* x8, const void* sx, const void* qweight, co
 
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group) {
   if (M <= 0 || M > kMaxM || check_kn(K, N, group) != AWQ_OK) return 0;
-  if (M > g_gemv_limit) return 1;
+  if (M > g_gemv_limit) return plan_gemm(M, K, N, sm_count_or_default()).stream_k ? 2 : 1;
   return plan_gemv(M, K, N, group, sm_count_or_default()).has_split ? 2 : 1;
 }
 

@@ -36,8 +36,10 @@ __host__ __device__ __forceinline__ int64_t block_index(int64_t nb, int64_t kb, 
 
 // Workspace layout (bytes):
 //   [0, 256)                   header: uint32 status word at offset 0
-//   [partial_off, ws_bytes)    decode GEMV fp32 partial sums of row blocks split
-//                              between CTAs: [ctas][2][8][16][M]
+//   [partial_off, ws_bytes)    decode GEMV (M <= 32): fp32 partial sums of row
+//                              blocks split between CTAs, [ctas][2][8][16][M];
+//                              stream-K GEMM (M > 32): fp32 parts of tiles split
+//                              between CTAs, [ctas][2][bn][128]
 constexpr size_t kWsHeaderBytes = 256;
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -73,6 +75,19 @@ struct GemvPlan {
 };
 GemvPlan plan_gemv(int64_t M, int64_t K, int64_t N, int group, int sm_count);
 
+// W4A16 GEMM schedule (shared by awq_workspace_bytes and the launcher).
+struct GemmPlan {
+  int bn;               // token tile (128 or 256)
+  int tiles;            // tiles of 128 channels x bn tokens
+  int gm;               // token tiles per block of the tile order
+  int ctas;             // persistent CTAs (at most one per SM)
+  int dp_tiles;         // the first dp_tiles tiles are computed whole, data-parallel
+  bool stream_k;        // the other tiles' k-blocks are split over the CTAs; the fixup kernel runs
+  size_t partial_off;   // workspace offset of the split tiles' fp32 parts (bytes)
+  size_t ws_bytes;      // total workspace bytes
+};
+GemmPlan plan_gemm(int64_t M, int64_t K, int64_t N, int sm_count);
+
 // Launchers (argument checks are done by the ABI layer).
 cudaError_t launch_pack(const __half* w, int64_t K, int64_t N, int group, uint32_t* qweight, __half* scales,
                         uint8_t* zeros, uint32_t* status, cudaStream_t stream);
@@ -82,8 +97,8 @@ cudaError_t launch_gemv(const __half* x, const uint32_t* qweight, const __half* 
                         __half* y, int64_t M, int64_t K, int64_t N, void* workspace, const GemvPlan& plan,
                         cudaStream_t stream);
 cudaError_t launch_gemm(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
-                        __half* y, int64_t M, int64_t K, int64_t N, int group, uint32_t* status,
-                        cudaStream_t stream);
+                        __half* y, int64_t M, int64_t K, int64_t N, int group, const GemmPlan& plan,
+                        void* workspace, cudaStream_t stream);
 
 // W4A8-FP8 variant (gemm_fp8.cu).
 cudaError_t launch_fp8_row_exponents(const __half* scales, int64_t K, int64_t N, int group, int8_t* e_out,

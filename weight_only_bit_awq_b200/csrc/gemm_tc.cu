@@ -106,6 +106,16 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, __half2 zlo, __half2 z
   return o;
 }
 
+// Tile order: blocks of GM token tiles; within a block, token tile fastest,
+// then channel tile. The x of one block stays in L2 while the block's channel
+// tiles stream past it.
+__device__ __forceinline__ void tile_coords(int t, int MT, int NT, int GM, int& mt, int& nt) {
+  const int blk = t / (GM * NT), w = t - blk * GM * NT;
+  const int gb = min(GM, MT - blk * GM);  // token tiles in this block
+  mt = blk * GM + w % gb;
+  nt = w / gb;
+}
+
 // GS: group size (128, 64 or 32), kGPK = 128 / GS groups per k-block.
 // Persistent: CTA c computes tiles c, c + P, c + 2P, ... (P = gridDim.x; tile
 // t is token tile t % MT of channel tile t / MT, so the CTAs running at the
@@ -116,7 +126,7 @@ template <int BN, int GS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
                 const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M,
-                int K, int N, int GM, uint32_t* status) {
+                int K, int N, int GM, int Tdp, float* __restrict__ partial, uint32_t* status) {
   using L = Layout<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -128,28 +138,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = K / kKPerBlock;
   const int MT = (M + BN - 1) / BN, NT = (N + kBM - 1) / kBM, T = MT * NT;
-  const int P = gridDim.x;
-  const int ntiles = blockIdx.x < T ? (T - 1 - (int)blockIdx.x) / P + 1 : 0;  // tiles of this CTA
-  // Tile order: blocks of GM token tiles; within a block, token tile fastest,
-  // then channel tile. The x of one block stays in L2 while the block's
-  // channel tiles stream past it.
-  auto tile_mn = [&](int it, int& mt, int& nt) {
-    const int t = (int)blockIdx.x + it * P;
-    const int blk = t / (GM * NT), w = t - blk * GM * NT;
-    const int gb = min(GM, MT - blk * GM);  // token tiles in this block
-    mt = blk * GM + w % gb;
-    nt = w / gb;
+  const int P = gridDim.x, c = blockIdx.x;
+  // Segments of this CTA: (tile t, k-blocks kb0 .. kb1 - 1). The first ndp are
+  // the whole tiles c, c + P, ... below Tdp; the rest cover this CTA's equal
+  // share [ub, ue) of the k-blocks of the last T - Tdp tiles ("stream-K"),
+  // which the fixup kernel adds up where a tile is split between CTAs.
+  const int ndp = c < Tdp ? (Tdp - 1 - c) / P + 1 : 0;
+  const int Usk = (T - Tdp) * KB;
+  const int ub = (int)((int64_t)c * Usk / P), ue = (int)((int64_t)(c + 1) * Usk / P);
+  const int nseg = ndp + (ub < ue ? (ue - 1) / KB - ub / KB + 1 : 0);
+  auto seg = [&](int j, int& t, int& kb0, int& kb1) {
+    if (j < ndp) {
+      t = c + j * P, kb0 = 0, kb1 = KB;
+    } else {
+      const int s = ub / KB + (j - ndp);
+      t = Tdp + s;
+      kb0 = j == ndp ? ub - s * KB : 0;
+      kb1 = min(KB, ue - s * KB);
+    }
   };
-  auto tile_m0 = [&](int it) {
-    int mt, nt;
-    tile_mn(it, mt, nt);
-    return mt * BN;
-  };
-  auto tile_nt = [&](int it) {
-    int mt, nt;
-    tile_mn(it, mt, nt);
-    return nt;
-  };
+  auto tile_mn = [&](int t, int& mt, int& nt) { tile_coords(t, MT, NT, GM, mt, nt); };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kXStages; ++i) {
@@ -184,15 +192,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  ptx::griddep_launch_dependents();  // lets the fixup kernel's CTAs become resident and wait
 
   if (warp == kWarpX) {
     // ---------------- x producer: 2 boxes of 64 k per k-block ----------------
     if (lane == 0) {
       int i = 0;  // stage uses so far
       bool ok = true;
-      for (int it = 0; it < ntiles && ok; ++it) {
-        const int m0 = tile_m0(it);
-        for (int h = 0; h < 2 * KB; ++h, ++i) {
+      for (int j = 0; j < nseg && ok; ++j) {
+        int t, kb0, kb1, mt, nt;
+        seg(j, t, kb0, kb1);
+        tile_mn(t, mt, nt);
+        const int m0 = mt * BN;
+        for (int h = 2 * kb0; h < 2 * kb1; ++h, ++i) {
           const int s = i % kXStages;
           if (!(ok = wait_bar(bar(kBarXEmpty + s), ((i / kXStages) & 1) ^ 1, abort_flag, status))) break;
           ptx::mbar_arrive_expect_tx(bar(kBarXFull + s), L::kXBytes);
@@ -213,11 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t NB = N / kRowsPerBlock;
     int i = 0;
     bool ok = true;
-    for (int it = 0; it < ntiles && ok; ++it) {
-      const int64_t gi = tile_nt(it);
+    for (int j = 0; j < nseg && ok; ++j) {
+      int t, kb0, kb1, mt, nt;
+      seg(j, t, kb0, kb1);
+      tile_mn(t, mt, nt);
+      const int64_t gi = nt;
       const int n0 = (int)gi * kBM;
       const uint32_t qbytes = (uint32_t)(group_rows(gi, NB) * 1024);
-      for (int kb = 0; kb < KB; ++kb, ++i) {
+      for (int kb = kb0; kb < kb1; ++kb, ++i) {
         const int s = i % kQStages;
         if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((i / kQStages) & 1) ^ 1, abort_flag, status);
         if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
@@ -250,12 +265,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = ptx::idesc_f16_f32(kBM, BN);
       bool ok = true;
       int wi = 0, xi = 0;  // W and x stage uses so far
-      for (int it = 0; it < ntiles && ok; ++it) {
-        const int acc = it & 1;
+      for (int j = 0; j < nseg && ok; ++j) {
+        int t, kb0, kb1;
+        seg(j, t, kb0, kb1);
+        const int acc = j & 1;
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);  // column offset of this accumulator
-        if (!(ok = wait_bar(bar(kBarAccEmpty + acc), ((it >> 1) & 1) ^ 1, abort_flag, status))) break;
+        if (!(ok = wait_bar(bar(kBarAccEmpty + acc), ((j >> 1) & 1) ^ 1, abort_flag, status))) break;
         ptx::tc_fence_after();
-        for (int kb = 0; kb < KB && ok; ++kb, ++wi) {
+        for (int kb = kb0; kb < kb1 && ok; ++kb, ++wi) {
           const int ws = wi % kWStages;
           if (!(ok = wait_bar(bar(kBarWFull + ws), (wi / kWStages) & 1, abort_flag, status))) break;
           ptx::tc_fence_after();
@@ -268,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               ptx::mma_f16_ss(d_tmem, ptx::desc_kmajor_sw128(a_base + 32 * kk),
-                              ptx::desc_kmajor_sw128(b_base + 32 * kk), idesc, (kb | h | kk) != 0);
+                              ptx::desc_kmajor_sw128(b_base + 32 * kk), idesc, ((kb - kb0) | h | kk) != 0);
             ptx::mma_commit(bar(kBarXEmpty + s));
           }
           if (ok) ptx::mma_commit(bar(kBarWEmpty + ws));
@@ -293,8 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kGPK = kKPerBlock / GS;
     bool ok = true;
     int i = 0;  // k-blocks so far (Q and W stage uses)
-    for (int it = 0; it < ntiles && ok; ++it) {
-      for (int kb = 0; kb < KB; ++kb, ++i) {
+    for (int j = 0; j < nseg && ok; ++j) {
+      int t, kb0, kb1;
+      seg(j, t, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb, ++i) {
         const int qs = i % kQStages;
         if (!(ok = wait_bar(bar(kBarQFull + qs), (i / kQStages) & 1, abort_flag, status))) break;
         const uint8_t* qst = smem + L::kQOff + qs * kQStride;
@@ -347,23 +366,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue: accumulator -> fp16 y ----------------
     const int quad = warp & 3;  // this warp may read TMEM lanes 32*quad .. +31
     const int r = 32 * quad + lane;
-    for (int it = 0; it < ntiles; ++it) {
-      const int acc = it & 1;
-      if (!wait_bar(bar(kBarAccFull + acc), (it >> 1) & 1, abort_flag, status)) break;
+    for (int j = 0; j < nseg; ++j) {
+      int t, kb0, kb1, mt, nt;
+      seg(j, t, kb0, kb1);
+      tile_mn(t, mt, nt);
+      const int acc = j & 1;
+      if (!wait_bar(bar(kBarAccFull + acc), (j >> 1) & 1, abort_flag, status)) break;
       ptx::tc_fence_after();
-      const int m0 = tile_m0(it), nn = tile_nt(it) * kBM + r;
+      const int m0 = mt * BN, nn = nt * kBM + r;
+      const bool whole = kb0 == 0 && kb1 == KB;
+      // a part of a split tile goes to this CTA's slot: 0 for its first
+      // stream-K segment, 1 for its last; layout [column m][row r], fp32
+      float* slot = whole ? nullptr : partial + ((int64_t)(2 * c + (j == ndp ? 0 : 1)) * BN) * kBM + r;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = 0; c0 < BN; c0 += 16) {
         if (m0 + c0 >= M) break;
-        uint32_t v[32];
-        ptx::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * BN + c0), v);
+        uint32_t v[16];
+        ptx::tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * BN + c0), v);
         ptx::tmem_wait_ld();
-        if (nn < N) {
+        if (!whole) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int m = m0 + c0 + j;
+          for (int q = 0; q < 16; ++q) __stcg(slot + (c0 + q) * kBM, __uint_as_float(v[q]));
+        } else if (nn < N) {
+#pragma unroll
+          for (int q = 0; q < 16; q += 2) {
+            const int m = m0 + c0 + q;
             // two conversions in one instruction, each rounded to nearest even
-            const __half2 h = __floats2half2_rn(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+            const __half2 h = __floats2half2_rn(__uint_as_float(v[q]), __uint_as_float(v[q + 1]));
             if (m < M) y[(int64_t)m * N + nn] = __low2half(h);
             if (m + 1 < M) y[(int64_t)(m + 1) * N + nn] = __high2half(h);
           }
@@ -380,6 +409,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, 2 * BN);
   }
+}
+
+// Stream-K tiles split between CTAs: CTA (s, b) adds the parts of stream-K
+// tile s, token columns 32 b .. 32 b + 31, thread = channel row of the tile.
+// The contributors are the CTAs whose k-block ranges meet the tile's, in CTA
+// order (so y does not depend on timing); a contributor's part is in its
+// slot 0 if its range starts inside the tile (the tile is its first
+// stream-K segment) and in slot 1 otherwise (the tile is its last). Tiles
+// that one CTA covered whole were written by the GEMM itself.
+// Launched right behind the GEMM (programmatic dependent launch): its CTAs
+// wait for the GEMM's writes in griddepcontrol.wait.
+template <int BN>
+__global__ void __launch_bounds__(kBM) gemm_fixup_kernel(const float* __restrict__ partial, __half* __restrict__ y,
+                                                         int M, int N, int KB, int GM, int Tdp, int P) {
+  ptx::griddep_launch_dependents();
+  const int MT = (M + BN - 1) / BN, NT = (N + kBM - 1) / kBM;
+  const int64_t Usk = (int64_t)(MT * NT - Tdp) * KB;
+  const int s = blockIdx.x;
+  auto cta_of = [&](int64_t u) { return (int)(((u + 1) * P - 1) / Usk); };  // CTA whose range holds unit u
+  const int c_first = cta_of((int64_t)s * KB), c_last = cta_of((int64_t)(s + 1) * KB - 1);
+  if (c_first == c_last) return;
+  int mt, nt;
+  tile_coords(Tdp + s, MT, NT, GM, mt, nt);
+  const int mb = mt * BN + 32 * (int)blockIdx.y;  // first token of this CTA
+  const int r = threadIdx.x, n = nt * kBM + r;
+  if (mb >= M || n >= N) return;
+  const int mcount = min(32, M - mb);
+  ptx::griddep_wait();
+  float v[32];
+#pragma unroll
+  for (int q = 0; q < 32; ++q) v[q] = 0.f;
+  for (int cc = c_first; cc <= c_last; ++cc) {
+    const int which = (int64_t)cc * Usk / P >= (int64_t)s * KB ? 0 : 1;
+    const float* p = partial + ((int64_t)(2 * cc + which) * BN + 32 * blockIdx.y) * kBM + r;
+#pragma unroll
+    for (int q = 0; q < 32; ++q)
+      if (q < mcount) v[q] += __ldcg(p + q * kBM);
+  }
+#pragma unroll
+  for (int q = 0; q < 32; ++q)
+    if (q < mcount) y[(int64_t)(mb + q) * N + n] = __float2half_rn(v[q]);
 }
 
 // Token tiles per block of the tile order: as many as keep the block's x
@@ -406,7 +476,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 
 template <int BN, int GS>
 cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
-                      __half* y, int64_t M, int64_t K, int64_t N, uint32_t* status, cudaStream_t stream) {
+                      __half* y, int64_t M, int64_t K, int64_t N, const GemmPlan& p, void* workspace,
+                      cudaStream_t stream) {
   using L = Layout<BN>;
   auto encode = get_encode();
   if (!encode) return cudaErrorNotSupported;
@@ -429,33 +500,82 @@ cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* sc
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
   }
-  const int64_t tiles = ((M + BN - 1) / BN) * ((N + kBM - 1) / kBM);
-  const int ctas = (int)(tiles < device_info().sm_count ? tiles : device_info().sm_count);  // one per SM
-  gemm_kernel<BN, GS><<<ctas, kThreads, L::kAlloc, stream>>>(tx, qweight, scales, zeros, y, (int)M, (int)K, (int)N,
-                                                             token_tiles_per_block(M, K, BN, 2), status);
-  return cudaGetLastError();
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* partial = p.stream_k ? reinterpret_cast<float*>(ws + p.partial_off) : nullptr;
+  gemm_kernel<BN, GS><<<p.ctas, kThreads, L::kAlloc, stream>>>(tx, qweight, scales, zeros, y, (int)M, (int)K, (int)N,
+                                                               p.gm, p.dp_tiles, partial, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !p.stream_k) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.tiles - p.dp_tiles), (unsigned)(BN / 32));
+  cfg.blockDim = dim3(kBM);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_fixup_kernel<BN>, (const float*)partial, y, (int)M, (int)N, (int)(K / kKPerBlock),
+                            p.gm, p.dp_tiles, p.ctas);
 }
 
 template <int GS>
 cudaError_t launch_gs(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
-                      __half* y, int64_t M, int64_t K, int64_t N, uint32_t* status, cudaStream_t stream) {
-  // 256-token tiles unless they cannot give every SM a tile and 128-token
-  // tiles would give it more (e.g. K=14336, N=4096, M=512: 64 against 128 tiles)
-  const int64_t nt = (N + kBM - 1) / kBM;
-  if (M > 128 && ((M + 255) / 256 * nt >= device_info().sm_count || (M + 127) / 128 * nt <= (M + 255) / 256 * nt))
-    return launch_bn<256, GS>(x, qweight, scales, zeros, y, M, K, N, status, stream);
-  return launch_bn<128, GS>(x, qweight, scales, zeros, y, M, K, N, status, stream);
+                      __half* y, int64_t M, int64_t K, int64_t N, const GemmPlan& p, void* workspace,
+                      cudaStream_t stream) {
+  if (p.bn == 256) return launch_bn<256, GS>(x, qweight, scales, zeros, y, M, K, N, p, workspace, stream);
+  return launch_bn<128, GS>(x, qweight, scales, zeros, y, M, K, N, p, workspace, stream);
 }
 
 }  // namespace
 
+// Schedule of the W4A16 GEMM.
+// Token tile: 256 unless 256-token tiles cannot give every SM a tile and
+// 128-token tiles would give it more (e.g. K=14336, N=4096, M=512: 64 against
+// 128 tiles).
+// Data-parallel: min(tiles, SMs) CTAs walk whole tiles. When that leaves the
+// last wave of tiles very short (under 80 % of the SM-tile slots busy), the
+// schedule turns "stream-K": all but the last full wave and the partial one
+// stay data-parallel, and the k-blocks of the remaining tiles are split
+// evenly over one CTA per SM, so every SM gets the same number of k-blocks;
+// tiles split between CTAs are finished by the fixup kernel from fp32 parts in
+// the workspace (two slots of 128 x BN per CTA). Measured on B200, stream-K
+// gains 8 % where 3.03 waves of tiles would take 4 (K=4096, N=28672, M=512)
+// but loses up to 4 % at 1.73 or 12.1 waves: the parts and the fixup cost
+// about what the idle SMs did. It needs at least 8 k-blocks per CTA and is
+// not used for M <= AWQ_GEMV_MAX_M, so decode-sized workspaces stay what the
+// GEMV needs.
+GemmPlan plan_gemm(int64_t M, int64_t K, int64_t N, int sm_count) {
+  GemmPlan p{};
+  const int64_t nt = (N + kBM - 1) / kBM;
+  p.bn = (M > 128 && ((M + 255) / 256 * nt >= sm_count || (M + 127) / 128 * nt <= (M + 255) / 256 * nt)) ? 256 : 128;
+  const int64_t mt = (M + p.bn - 1) / p.bn, KB = K / kKPerBlock;
+  p.tiles = (int)(mt * nt);
+  p.gm = token_tiles_per_block(M, K, p.bn, 2);
+  p.ctas = p.tiles < sm_count ? p.tiles : sm_count;
+  p.dp_tiles = p.tiles;
+  p.ws_bytes = kWsHeaderBytes;
+  const int64_t waves = (p.tiles + sm_count - 1) / sm_count;
+  const int64_t tsk = p.tiles < sm_count ? p.tiles : sm_count + p.tiles % sm_count;
+  if (M > AWQ_GEMV_MAX_M && p.tiles % sm_count != 0 && 100 * (int64_t)p.tiles < 80 * waves * sm_count &&
+      tsk * KB >= 8 * (int64_t)sm_count) {
+    p.stream_k = true;
+    p.ctas = sm_count;
+    p.dp_tiles = (int)(p.tiles - tsk);
+    p.partial_off = kWsHeaderBytes;
+    p.ws_bytes = p.partial_off + (size_t)p.ctas * 2 * p.bn * kBM * sizeof(float);
+  }
+  return p;
+}
+
 cudaError_t launch_gemm(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
-                        __half* y, int64_t M, int64_t K, int64_t N, int group, uint32_t* status,
+                        __half* y, int64_t M, int64_t K, int64_t N, int group, const GemmPlan& plan, void* workspace,
                         cudaStream_t stream) {
   switch (group) {
-    case 128: return launch_gs<128>(x, qweight, scales, zeros, y, M, K, N, status, stream);
-    case 64: return launch_gs<64>(x, qweight, scales, zeros, y, M, K, N, status, stream);
-    case 32: return launch_gs<32>(x, qweight, scales, zeros, y, M, K, N, status, stream);
+    case 128: return launch_gs<128>(x, qweight, scales, zeros, y, M, K, N, plan, workspace, stream);
+    case 64: return launch_gs<64>(x, qweight, scales, zeros, y, M, K, N, plan, workspace, stream);
+    case 32: return launch_gs<32>(x, qweight, scales, zeros, y, M, K, N, plan, workspace, stream);
     default: return cudaErrorInvalidConfiguration;
   }
 }
