@@ -539,6 +539,7 @@ SINGLE = {
     # one kernel on a layer larger than the 126 MB L2, for profiler captures
     "gemv": ("llama2_70b_decode", "gate_up", 1),     # 235 MB packed weight, M = 1
     "gemm": ("prefill", "llama3_gate_up", 2048),     # 58 MB weight + 16 MB x + 117 MB y
+    "gemm_m512": ("prefill", "llama3_gate_up", 512),  # stream-K schedule: the GEMM and its fixup kernel
     "gemm_fp8": ("prefill", "llama3_gate_up", 2048),  # the same layer through the W4A8-FP8 GEMM
 }
 

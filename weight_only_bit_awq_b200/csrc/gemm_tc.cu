@@ -29,8 +29,11 @@
 //           sub-partition hide the dependent fp16 chains).
 //   warps 11-14 drain a finished accumulator (tcgen05.ld; warp w reads TMEM
 //           lanes 32 (w % 4) ..) into fp16 y and release it.
-// Rings: x 4 x (BN x 64 k), dequantized weight 2 x (128 x 128 k), packed
-// weight 3 x 8 KiB, each with full/empty mbarriers. Every wait is bounded
+// Rings: x 3 x (BN x 64 k) for BN = 256, 6 x for BN = 128; dequantized weight
+// 3 x (128 x 128 k); packed weight 3 x 8 KiB; each with full/empty mbarriers.
+// (Measured on B200: 3 + 3 stages beat 4 + 2 by ~1 %; two x stages lose 9 %;
+// 6-8 packed-weight stages or an L2 prefetch of the codes a few k-blocks
+// ahead gain nothing.) Every wait is bounded
 // (2 s of %globaltimer); on expiry the CTA records AWQ_ERR_TIMEOUT in the
 // status word, the other roles stop at their next wait, in-flight copies and
 // MMAs are drained, tensor memory is freed and the CTA exits.
@@ -45,8 +48,6 @@ namespace awq {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kXStages = 4;
-constexpr int kWStages = 2;
 constexpr int kQStages = 3;
 constexpr int kQBytes = 8 * 1024;
 // Behind a stage's codes: the tile's scale rows (up to 4 groups x 128 fp16)
@@ -60,14 +61,17 @@ constexpr int kFirstEpiWarp = kFirstDeqWarp + kNumDeqWarps, kNumEpiWarps = 4;
 constexpr int kDeqThreads = kNumDeqWarps * 32, kEpiThreads = kNumEpiWarps * 32;
 constexpr int kThreads = (kFirstEpiWarp + kNumEpiWarps) * 32;
 
-// barrier indices
-constexpr int kBarXFull = 0, kBarXEmpty = kBarXFull + kXStages, kBarWFull = kBarXEmpty + kXStages,
-              kBarWEmpty = kBarWFull + kWStages, kBarQFull = kBarWEmpty + kWStages,
-              kBarQEmpty = kBarQFull + kQStages, kBarAccFull = kBarQEmpty + kQStages, kBarAccEmpty = kBarAccFull + 2,
-              kBarDrain = kBarAccEmpty + 2, kNumBars = kBarDrain + 1;
-
 template <int BN>
 struct Layout {
+  // ring depths: x stages of 64 k (BN x 64 fp16), dequantized-weight stages
+  // of one 128-k block
+  static constexpr int kXStages = BN == 256 ? 3 : 6;
+  static constexpr int kWStages = 3;
+  // barrier indices
+  static constexpr int kBarXFull = 0, kBarXEmpty = kBarXFull + kXStages, kBarWFull = kBarXEmpty + kXStages,
+                       kBarWEmpty = kBarWFull + kWStages, kBarQFull = kBarWEmpty + kWStages,
+                       kBarQEmpty = kBarQFull + kQStages, kBarAccFull = kBarQEmpty + kQStages,
+                       kBarAccEmpty = kBarAccFull + 2, kBarDrain = kBarAccEmpty + 2, kNumBars = kBarDrain + 1;
   static constexpr int kXBytes = BN * 64 * 2;
   static constexpr int kXOff = 0;
   static constexpr int kWOff = kXOff + kXStages * kXBytes;
@@ -77,7 +81,7 @@ struct Layout {
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1 KiB
 };
-static_assert(Layout<256>::kAlloc <= 232448, "shared memory budget");
+static_assert(Layout<256>::kAlloc <= 232448 && Layout<128>::kAlloc <= 232448, "shared memory budget");
 
 using ptx::drain_bar;
 using ptx::wait_bar;
@@ -128,6 +132,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M,
                 int K, int N, int GM, int Tdp, float* __restrict__ partial, uint32_t* status) {
   using L = Layout<BN>;
+  constexpr int kXStages = L::kXStages, kWStages = L::kWStages;
+  constexpr int kBarXFull = L::kBarXFull, kBarXEmpty = L::kBarXEmpty, kBarWFull = L::kBarWFull,
+                kBarWEmpty = L::kBarWEmpty, kBarQFull = L::kBarQFull, kBarQEmpty = L::kBarQEmpty,
+                kBarAccFull = L::kBarAccFull, kBarAccEmpty = L::kBarAccEmpty, kBarDrain = L::kBarDrain;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
