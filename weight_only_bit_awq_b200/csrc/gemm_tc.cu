@@ -21,12 +21,12 @@
 //           stage barriers and, at the end of a tile, to its accumulator's.
 //   warp 2  issues bulk copies of the packed weight: the tile's 8 row blocks
 //           of one 128-k block are one contiguous 8 KiB run.
-//   warps 3-10 dequantize: threads 2r and 2r + 1 own weight row r of the
-//           tile, each reads half of its 64 B of codes for the k-block from
-//           shared memory, forms fp16_rne((q - z) * s) (the exact value the
-//           dequant kernel and the CPU oracle produce) and stores it,
-//           swizzled, into the A-operand buffer (two warps per SM
-//           sub-partition hide the dependent fp16 chains).
+//   warps 3-10 dequantize in two groups of four that take alternate
+//           k-blocks (two k-blocks in flight): in a group, thread r owns
+//           weight row r of the tile, reads its 64 B of codes for the k-block
+//           from shared memory, forms fp16_rne((q - z) * s) (the exact value
+//           the dequant kernel and the CPU oracle produce) and stores it,
+//           swizzled, into the A-operand buffer.
 //   warps 11-14 drain a finished accumulator (tcgen05.ld; warp w reads TMEM
 //           lanes 32 (w % 4) ..) into fp16 y and release it.
 // Rings: x 3 x (BN x 64 k) for BN = 256, 6 x for BN = 128; dequantized weight
@@ -173,13 +173,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(bar(kBarXEmpty + i), 1);
     }
     for (int i = 0; i < kWStages; ++i) {
-      ptx::mbar_init(bar(kBarWFull + i), kDeqThreads);
+      ptx::mbar_init(bar(kBarWFull + i), kDeqThreads / 2);  // one group of dequant warps fills a stage
       ptx::mbar_init(bar(kBarWEmpty + i), 1);
     }
     for (int i = 0; i < kQStages; ++i) {
       // the codes' byte count + 32 cp.async arrivals (scales, zeros)
       ptx::mbar_init(bar(kBarQFull + i), 33);
-      ptx::mbar_init(bar(kBarQEmpty + i), kDeqThreads);
+      ptx::mbar_init(bar(kBarQEmpty + i), kDeqThreads / 2);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bar(kBarAccFull + i), 1);
@@ -308,13 +308,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp < kFirstEpiWarp) {
     // ---------------- dequantize ----------------
-    // Thread d = (row, half): row = d / 2 takes words 8 half .. 8 half + 7 of
-    // its row, two 16-byte chunks read and stored in a rotated order (the
-    // rotation also depends on the half) so that every 8-lane phase of the
-    // shared loads and of the swizzled stores touches distinct banks.
+    // Two groups of four warps take alternate k-blocks, so two k-blocks are
+    // in flight and one group's barrier waits, loads and proxy fence overlap
+    // the other's arithmetic. In a group, thread = weight row: it reads the
+    // row's 64 B of codes as four 16-byte chunks in an order rotated by
+    // (row / 2) % 4, so that every 8-lane phase of the shared loads and of the
+    // swizzled stores touches distinct banks.
     const int d = threadIdx.x - kFirstDeqWarp * 32;  // 0..255
-    const int row = d >> 1, hf = d & 1;
-    const int rot = ((row >> 1) ^ hf) & 1;
+    const int grp = d >> 7, row = d & (kBM - 1);
+    const int rot = (row >> 1) & 3;
     constexpr int kGPK = kKPerBlock / GS;
     bool ok = true;
     int i = 0;  // k-blocks so far (Q and W stage uses)
@@ -322,13 +324,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t, kb0, kb1;
       seg(j, t, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb, ++i) {
+        if ((i & 1) != grp) continue;  // the other group's k-block
         const int qs = i % kQStages;
         if (!(ok = wait_bar(bar(kBarQFull + qs), (i / kQStages) & 1, abort_flag, status))) break;
         const uint8_t* qst = smem + L::kQOff + qs * kQStride;
-        const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64 + 32 * hf;
-        uint4 c[2];
+        const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64;
+        uint4 c[4];
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 1));
+        for (int jj = 0; jj < 4; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 3));
         // fp16 bits of the scale and the zero point of this row, per group (rows
         // past N read stale values: their outputs are never stored)
         uint32_t s[kGPK], z[kGPK];
@@ -351,8 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int cj = 2 * hf + ((jj + rot) & 1);  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
+        for (int jj = 0; jj < 4; ++jj) {
+          const int cj = (jj + rot) & 3;  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
           const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
 #pragma unroll
           for (int ww = 0; ww < 4; ++ww) {
