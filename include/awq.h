@@ -67,7 +67,8 @@
  *   Workspace  at least awq_workspace_bytes(M, K, N, group) bytes of device
  *              memory, zeroed once with awq_workspace_init before first use.
  *              Only its status word must start at zero; the GEMV's partial
- *              sums of split rows are written before they are read. One
+ *              sums of split rows and the GEMM's stream-K parts of split
+ *              tiles are written before they are read. One
  *              workspace must not be used by two calls that can run at the
  *              same time (e.g. on two streams).
  */
@@ -107,8 +108,11 @@ typedef struct awq_packed_sizes {
 awq_status awq_packed_size(int64_t K, int64_t N, int group, awq_packed_sizes* out);
 
 /* Workspace bytes needed by any entry point below for these sizes on the
- * current device (the status word, the GEMV's partial sums of rows split between CTAs). Host only.
- * Returns 0 for invalid sizes. */
+ * current device: the status word, plus for 1 <= M <= AWQ_GEMV_MAX_M the
+ * GEMV's partial sums of rows split between CTAs, and for M > AWQ_GEMV_MAX_M,
+ * when the GEMM's schedule is stream-K, its fp32 parts of split tiles (two
+ * slots of 128 x 256 floats per SM at most). Host only. Returns 0 for invalid
+ * sizes. */
 size_t awq_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
 
 /* Zero `ws_bytes` bytes of workspace on `stream` (needed once, before the
