@@ -121,11 +121,14 @@ __device__ __forceinline__ void tile_coords(int t, int MT, int NT, int GM, int& 
 }
 
 // GS: group size (128, 64 or 32), kGPK = 128 / GS groups per k-block.
-// Persistent: CTA c computes tiles c, c + P, c + 2P, ... (P = gridDim.x; tile
-// t is token tile t % MT of channel tile t / MT, so the CTAs running at the
-// same time share a few weight tiles). Every role walks the same tile
-// sequence; the rings run on across tile boundaries, and the two accumulators
-// let the epilogue warps drain tile j while the MMA warp fills tile j + 1.
+// Persistent: CTA c computes the whole tiles c, c + P, c + 2P, ... below Tdp
+// (P = gridDim.x; tile t maps to (token tile, channel tile) by tile_coords, so
+// the CTAs running at the same time share a few weight tiles), then its share
+// of the k-blocks of tiles Tdp .. T - 1 (stream-K; none when Tdp = T). Every
+// role walks the same segment sequence; the rings run on across segment
+// boundaries, and the two accumulators let the epilogue warps drain segment j
+// while the MMA warp fills segment j + 1. `partial` (the workspace slots of
+// split tiles) is only used when Tdp < T.
 template <int BN, int GS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
