@@ -37,6 +37,7 @@
 // (2 s of %globaltimer); on expiry the CTA records AWQ_ERR_TIMEOUT in the
 // status word, the other roles stop at their next wait, in-flight copies and
 // MMAs are drained, tensor memory is freed and the CTA exits.
+#include <atomic>
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -48,7 +49,6 @@ namespace awq {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kQStages = 3;
 constexpr int kQBytes = 8 * 1024;
 // Behind a stage's codes: the tile's scale rows (up to 4 groups x 128 fp16)
 // and zero-point rows (up to 4 x 64 bytes) of that k-block.
@@ -64,9 +64,12 @@ constexpr int kThreads = (kFirstEpiWarp + kNumEpiWarps) * 32;
 template <int BN>
 struct Layout {
   // ring depths: x stages of 64 k (BN x 64 fp16), dequantized-weight stages
-  // of one 128-k block
-  static constexpr int kXStages = BN == 256 ? 3 : 6;
+  // of one 128-k block, code stages (an even number: the two dequant groups
+  // take alternate k-blocks, and each stage must belong to one group)
+  static constexpr int kXStages = BN == 256 ? 3 : 5;
   static constexpr int kWStages = 3;
+  static constexpr int kQStages = BN == 256 ? 2 : 4;
+  static_assert(kQStages % 2 == 0, "each code stage belongs to one dequant group");
   // barrier indices
   static constexpr int kBarXFull = 0, kBarXEmpty = kBarXFull + kXStages, kBarWFull = kBarXEmpty + kXStages,
                        kBarWEmpty = kBarWFull + kWStages, kBarQFull = kBarWEmpty + kWStages,
@@ -133,9 +136,9 @@ template <int BN, int GS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
                 const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M,
-                int K, int N, int GM, int Tdp, float* __restrict__ partial, uint32_t* status) {
+                int K, int N, int GM, int Tdp, float* __restrict__ partial, int64_t part_floats, uint32_t* status) {
   using L = Layout<BN>;
-  constexpr int kXStages = L::kXStages, kWStages = L::kWStages;
+  constexpr int kXStages = L::kXStages, kWStages = L::kWStages, kQStages = L::kQStages;
   constexpr int kBarXFull = L::kBarXFull, kBarXEmpty = L::kBarXEmpty, kBarWFull = L::kBarWFull,
                 kBarWEmpty = L::kBarWEmpty, kBarQFull = L::kBarQFull, kBarQEmpty = L::kBarQEmpty,
                 kBarAccFull = L::kBarAccFull, kBarAccEmpty = L::kBarAccEmpty, kBarDrain = L::kBarDrain;
@@ -248,18 +251,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((i / kQStages) & 1) ^ 1, abort_flag, status);
         if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
         const uint32_t st = sbase + L::kQOff + s * kQStride;
-        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qbytes);
+        const int64_t qw0 = unit_first_block(gi, kb, KB, NB) * kWordsPerBlock;
+        const bool qok = AWQ_CHECK(in_range(qw0, qbytes / 4, (int64_t)K * N / 8), status);
+        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qok ? qbytes : 0u);
         __syncwarp();
-        if (lane == 0)
-          ptx::bulk_g2s(st, qweight + unit_first_block(gi, kb, KB, NB) * kWordsPerBlock, qbytes, bar(kBarQFull + s));
+        if (lane == 0 && qok) ptx::bulk_g2s(st, qweight + qw0, qbytes, bar(kBarQFull + s));
         for (int p = lane; p < kGPK * 16; p += 32) {  // kGPK rows of 128 scales: 16 B = 8 output channels
           const int g = p >> 4, l = p & 15;
-          if (n0 + 8 * l < N)
+          if (n0 + 8 * l < N &&
+              AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * N + n0 + 8 * l, 8, (int64_t)(K / GS) * N), status))
             ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
         }
         for (int p = lane; p < kGPK * 8; p += 32) {  // kGPK rows of 64 zero bytes: 8 B = 16 output channels
           const int g = p >> 3, l = p & 7;
-          if (n0 + 16 * l < N)
+          if (n0 + 16 * l < N &&
+              AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l, 8, (int64_t)(K / GS) * (N / 2)),
+                        status))
             ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l,
                             zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
         }
@@ -328,6 +335,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       seg(j, t, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb, ++i) {
         if ((i & 1) != grp) continue;  // the other group's k-block
+        // kQStages is even, so stage qs = i % kQStages always belongs to this
+        // group and its uses reach this group in order, one phase apart (an
+        // odd ring shared by alternating groups let a group wait two phases
+        // ahead of a stage whose previous use had not landed, and a parity
+        // wait cannot tell those phases apart)
         const int qs = i % kQStages;
         if (!(ok = wait_bar(bar(kBarQFull + qs), (i / kQStages) & 1, abort_flag, status))) break;
         const uint8_t* qst = smem + L::kQOff + qs * kQStride;
@@ -399,16 +411,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * BN + c0), v);
         ptx::tmem_wait_ld();
         if (!whole) {
+          if (AWQ_CHECK(in_range(slot - partial + c0 * kBM, 15 * kBM + 1, part_floats), status)) {
 #pragma unroll
-          for (int q = 0; q < 16; ++q) __stcg(slot + (c0 + q) * kBM, __uint_as_float(v[q]));
+            for (int q = 0; q < 16; ++q) __stcg(slot + (c0 + q) * kBM, __uint_as_float(v[q]));
+          }
         } else if (nn < N) {
 #pragma unroll
           for (int q = 0; q < 16; q += 2) {
             const int m = m0 + c0 + q;
             // two conversions in one instruction, each rounded to nearest even
             const __half2 h = __floats2half2_rn(__uint_as_float(v[q]), __uint_as_float(v[q + 1]));
-            if (m < M) y[(int64_t)m * N + nn] = __low2half(h);
-            if (m + 1 < M) y[(int64_t)(m + 1) * N + nn] = __high2half(h);
+            if (m < M && AWQ_CHECK(in_range((int64_t)m * N + nn, 1, (int64_t)M * N), status))
+              y[(int64_t)m * N + nn] = __low2half(h);
+            if (m + 1 < M && AWQ_CHECK(in_range((int64_t)(m + 1) * N + nn, 1, (int64_t)M * N), status))
+              y[(int64_t)(m + 1) * N + nn] = __high2half(h);
           }
         }
       }
@@ -436,7 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // wait for the GEMM's writes in griddepcontrol.wait.
 template <int BN>
 __global__ void __launch_bounds__(kBM) gemm_fixup_kernel(const float* __restrict__ partial, __half* __restrict__ y,
-                                                         int M, int N, int KB, int GM, int Tdp, int P) {
+                                                         int M, int N, int KB, int GM, int Tdp, int P,
+                                                         int64_t part_floats, uint32_t* status) {
   ptx::griddep_launch_dependents();
   const int MT = (M + BN - 1) / BN, NT = (N + kBM - 1) / kBM;
   const int64_t Usk = (int64_t)(MT * NT - Tdp) * KB;
@@ -457,10 +474,12 @@ __global__ void __launch_bounds__(kBM) gemm_fixup_kernel(const float* __restrict
   for (int cc = c_first; cc <= c_last; ++cc) {
     const int which = (int64_t)cc * Usk / P >= (int64_t)s * KB ? 0 : 1;
     const float* p = partial + ((int64_t)(2 * cc + which) * BN + 32 * blockIdx.y) * kBM + r;
+    if (!AWQ_CHECK(in_range(p - partial, (int64_t)(mcount - 1) * kBM + 1, part_floats), status)) return;
 #pragma unroll
     for (int q = 0; q < 32; ++q)
       if (q < mcount) v[q] += __ldcg(p + q * kBM);
   }
+  if (!AWQ_CHECK(in_range((int64_t)mb * N + n, (int64_t)(mcount - 1) * N + 1, (int64_t)M * N), status)) return;
 #pragma unroll
   for (int q = 0; q < 32; ++q)
     if (q < mcount) y[(int64_t)(mb + q) * N + n] = __float2half_rn(v[q]);
@@ -506,19 +525,20 @@ cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* sc
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  static uint64_t attr_set = 0;  // one bit per device that has the attribute
+  static std::atomic<uint64_t> attr_set{0};  // one bit per device that has the attribute
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
-  if (!(attr_set >> dev & 1)) {
+  if (!(attr_set.load(std::memory_order_acquire) >> dev & 1)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
-    attr_set |= uint64_t(1) << dev;
+    attr_set.fetch_or(uint64_t(1) << dev, std::memory_order_acq_rel);
   }
   char* ws = static_cast<char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   float* partial = p.stream_k ? reinterpret_cast<float*>(ws + p.partial_off) : nullptr;
+  const int64_t part_floats = p.stream_k ? (int64_t)(p.ws_bytes - p.partial_off) / 4 : 0;
   gemm_kernel<BN, GS><<<p.ctas, kThreads, L::kAlloc, stream>>>(tx, qweight, scales, zeros, y, (int)M, (int)K, (int)N,
-                                                               p.gm, p.dp_tiles, partial, status);
+                                                               p.gm, p.dp_tiles, partial, part_floats, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !p.stream_k) return e;
   cudaLaunchConfig_t cfg = {};
@@ -531,7 +551,7 @@ cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* sc
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, gemm_fixup_kernel<BN>, (const float*)partial, y, (int)M, (int)N, (int)(K / kKPerBlock),
-                            p.gm, p.dp_tiles, p.ctas);
+                            p.gm, p.dp_tiles, p.ctas, part_floats, status);
 }
 
 template <int GS>
