@@ -59,6 +59,12 @@
  *              only per-device launch parameters (SM count, kernel attributes).
  *   Streams    `stream` is a cudaStream_t (NULL = legacy default stream).
  *              Calls are asynchronous on it; only awq_get_status synchronizes.
+ *   Debug      the library built with -DAWQ_DEBUG (weight_only_bit_awq_b200/
+ *              build.py --debug: libawq_b200_debug.so, same entry points)
+ *              checks the index range of every global and shared access of
+ *              the pack, dequant, GEMV and GEMM kernels before it happens; a
+ *              failed check records AWQ_ERR_BOUNDS in the status word and
+ *              skips the access instead of faulting.
  *   Errors     argument errors are returned before anything is launched;
  *              AWQ_ERR_CUDA reports a failed launch. Errors found on the device
  *              (a non-finite weight in awq_pack, a bounded wait that expired)
@@ -91,7 +97,8 @@ typedef enum awq_status {
   AWQ_ERR_UNSUPPORTED = 5, /* group not 32, 64 or 128, M above an entry's limit, no sm_100 device */
   AWQ_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed */
   AWQ_ERR_TIMEOUT = 7,     /* device side: a bounded pipeline wait expired */
-  AWQ_ERR_NONFINITE = 8    /* device side: awq_pack met an inf or NaN weight */
+  AWQ_ERR_NONFINITE = 8,   /* device side: awq_pack met an inf or NaN weight */
+  AWQ_ERR_BOUNDS = 9       /* device side, debug build only: an index check failed (the access was skipped) */
 } awq_status;
 
 typedef struct awq_packed_sizes {
@@ -104,30 +111,40 @@ typedef struct awq_packed_sizes {
 #define AWQ_GEMV_MAX_M 32
 
 /* Sizes of the three packed buffers for a [N][K] weight. Host only.
- * Returns AWQ_ERR_SHAPE / AWQ_ERR_UNSUPPORTED / AWQ_ERR_INVALID_ARG (out NULL). */
+ * Returns AWQ_ERR_SHAPE / AWQ_ERR_UNSUPPORTED / AWQ_ERR_INVALID_ARG (out NULL).
+ * Source: TinyChat README, Usage step 3 (4-bit codes per group of 128
+ * inputs); the byte counts follow from the packed layout above. */
 awq_status awq_packed_size(int64_t K, int64_t N, int group, awq_packed_sizes* out);
 
 /* Workspace bytes needed by any entry point below for these sizes on the
- * current device: the status word, plus for 1 <= M <= AWQ_GEMV_MAX_M the
- * GEMV's partial sums of rows split between CTAs, and for M > AWQ_GEMV_MAX_M,
- * when the GEMM's schedule is stream-K, its fp32 parts of split tiles (two
- * slots of 128 x 256 floats per SM at most). Host only. Returns 0 for invalid
- * sizes. */
+ * current device: the status word, plus, when the decode GEMV's plan splits
+ * rows between CTAs, its partial sums of those rows, and for M >
+ * AWQ_GEMV_MAX_M, when the GEMM's schedule is stream-K, its fp32 parts of
+ * split tiles (two slots of 128 x 256 floats per SM at most). Host only.
+ * Returns 0 for invalid sizes.
+ * Source: none on the pages (the kernels' scratch memory, owned by the caller). */
 size_t awq_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
 
 /* Zero `ws_bytes` bytes of workspace on `stream` (needed once, before the
- * first use of a new workspace). */
+ * first use of a new workspace).
+ * Source: none on the pages (workspace set-up). */
 awq_status awq_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
 /* Quantize and pack (TinyChat README, Usage step 3: "--w_bit 4
  * --q_group_size 128 ... --q_backend real"): W fp16 [N][K] -> qweight,
  * scales, zeros in the layout above, bit for bit the quantization stated
  * above. An inf/NaN weight records AWQ_ERR_NONFINITE in the workspace status
- * word (its group's outputs are then unspecified). */
+ * word (its group's outputs are then unspecified).
+ * Source: TinyChat README, Usage step 3 (the quantization knobs). */
 awq_status awq_pack(const void* w, int64_t K, int64_t N, int group, void* qweight, void* scales, void* zeros,
                     void* workspace, size_t ws_bytes, void* stream);
 
-/* Dequantize: W^ fp16 [N][K] = fp16_rne((q - z) * s) for every (n, k). */
+/* Dequantize: W^ fp16 [N][K] = fp16_rne((q - z) * s) for every (n, k). The
+ * bit-exact test surface of the packed format; w_out must not overlap the
+ * packed buffers.
+ * Source: TinyChat README, Usage step 3 (the 4-bit weights with a scale and
+ * zero point per group, "--q_backend real" storing them packed); w = (q - z) s
+ * is the asymmetric reading stated at the top of this header. */
 awq_status awq_dequant(const void* qweight, const void* scales, const void* zeros, int64_t K, int64_t N,
                        int group, void* w_out, void* stream);
 
@@ -139,7 +156,8 @@ awq_status awq_dequant(const void* qweight, const void* scales, const void* zero
  * 128-input block's largest magnitude). Rows whose k-range is split between
  * CTAs are added in a fixed order, so results are deterministic. A non-finite
  * x[m][k] gives non-finite y[m][*]. M > AWQ_GEMV_MAX_M returns
- * AWQ_ERR_UNSUPPORTED. */
+ * AWQ_ERR_UNSUPPORTED.
+ * Source: TinyChat README, Speed Benchmarks (per-token generation latency). */
 awq_status awq_w4a16_gemv(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
                           int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,
                           void* stream);
@@ -151,13 +169,19 @@ awq_status awq_w4a16_gemv(const void* x, const void* qweight, const void* scales
  * tiles would leave the last wave of SMs short, the k-range of the last tiles
  * is split between CTAs ("stream-K") and a second kernel adds the fp32 parts,
  * which live in the workspace, in a fixed order: results are deterministic
- * for a given device (SM count). */
+ * for a given device (SM count).
+ * Source: TinyChat README, New Optimization of Context Stage. */
 awq_status awq_w4a16_gemm(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
                           int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,
                           void* stream);
 
-/* The linear layer: awq_w4a16_gemv for M <= awq_linear_gemv_limit(), else
- * awq_w4a16_gemm. */
+/* The linear layer: awq_w4a16_gemv for M <= awq_linear_gemv_limit() (16),
+ * and for 16 < M <= AWQ_GEMV_MAX_M when the layer has fewer 128-channel tiles
+ * than the device has SMs (ceil(N / 128) < SMs); awq_w4a16_gemm otherwise.
+ * The split was measured on B200: the GEMV wins every decode layer up to
+ * M = 16, the GEMM wins the wide layers from M = 24.
+ * Source: TinyChat README, Speed Benchmarks and New Optimization of Context
+ * Stage (the same W4A16 linear layers at decode and at prefill). */
 awq_status awq_linear(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
                       int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,
                       void* stream);
@@ -183,17 +207,20 @@ awq_status awq_linear(const void* x, const void* qweight, const void* scales, co
 
 /* e[n] (int8, one per output channel) from the packed scales fp16 [K/group][N]
  * as awq_pack wrote them (positive). Shapes and group as for every entry
- * point; scales 16-byte aligned; e_out any alignment, not overlapping scales. */
+ * point; scales 16-byte aligned; e_out any alignment, not overlapping scales.
+ * Source: TensorRT-LLM news item on INT4 AWQ on one H200 (FP8 compute). */
 awq_status awq_fp8_row_exponents(const void* scales, int64_t K, int64_t N, int group, void* e_out, void* stream);
 
 /* x fp16 [M][K] -> x8 E4M3 codes uint8 [M][K] and sx fp32 [M] (formulas above).
  * K % 128 == 0; M >= 0 (0 is a no-op); x, x8 and sx 16-byte aligned and not
  * overlapping. A row holding inf or NaN gives codes and sx that are not
- * finite numbers (NaN, or 0 codes with sx = inf). */
+ * finite numbers (NaN, or 0 codes with sx = inf).
+ * Source: TensorRT-LLM news item on INT4 AWQ on one H200 (FP8 compute). */
 awq_status awq_fp8_quantize_x(const void* x, int64_t M, int64_t K, void* x8, void* sx, void* stream);
 
 /* W8 uint8 [N][K] = the E4M3 codes the W4A8 GEMM multiplies (test surface,
- * like awq_dequant): row_exp is e from awq_fp8_row_exponents. */
+ * like awq_dequant): row_exp is e from awq_fp8_row_exponents.
+ * Source: TensorRT-LLM news item on INT4 AWQ on one H200 (FP8 compute). */
 awq_status awq_dequant_fp8(const void* qweight, const void* scales, const void* zeros, const void* row_exp,
                            int64_t K, int64_t N, int group, void* w8_out, void* stream);
 
@@ -203,12 +230,15 @@ awq_status awq_dequant_fp8(const void* qweight, const void* scales, const void* 
  * dequantized to E4M3 in shared memory just ahead of the MMA. Any M >= 0.
  * x8, sx, y, the packed buffers and the workspace 16-byte aligned; y must not
  * overlap any input. The workspace needs only its status word
- * (ws_bytes >= 256); an expired bounded wait records AWQ_ERR_TIMEOUT there. */
+ * (ws_bytes >= 256); an expired bounded wait records AWQ_ERR_TIMEOUT there.
+ * Source: TensorRT-LLM news item on INT4 AWQ on one H200 (FP8 compute). */
 awq_status awq_w4a8_gemm(const void* x8, const void* sx, const void* qweight, const void* scales, const void* zeros,
                          const void* row_exp, void* y, int64_t M, int64_t K, int64_t N, int group, void* workspace,
                          size_t ws_bytes, void* stream);
 
-/* The M at and below which awq_linear takes the GEMV path. */
+/* The M at and below which awq_linear always takes the GEMV path (above it,
+ * up to AWQ_GEMV_MAX_M, only for layers with fewer 128-channel tiles than SMs).
+ * Source: none on the pages (a dispatch threshold set from measurements). */
 int awq_linear_gemv_limit(void);
 
 /* Size of the library-owned scratch array behind awq_w4a16_gemv_no_alloc:
@@ -229,14 +259,26 @@ int awq_linear_gemv_limit(void);
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture. Every call uses the same array: calls that can
  * overlap on the GPU race on it. Each call zeroes the status word (a memset
- * on `stream`) before its kernels run. */
+ * on `stream`) before its kernels run.
+ * Source: none on the pages (an allocation-free variant for such callers). */
 awq_status awq_w4a16_gemv_no_alloc(const void* x, const void* qweight, const void* scales, const void* zeros,
                                    void* y, int64_t M, int64_t K, int64_t N, int group, void* stream);
 
+/* The device-side status word of awq_w4a16_gemv_no_alloc's scratch array on
+ * the current device: synchronize `stream`, then return and clear it (AWQ_OK
+ * if nothing was recorded; AWQ_ERR_TIMEOUT if a bounded wait of the GEMV
+ * expired). Like the workspace status of awq_get_status, a device-side error
+ * is only seen here, so call it after the calls whose outcome matters and
+ * before the next awq_w4a16_gemv_no_alloc, which clears the word again.
+ * Allocates nothing. AWQ_ERR_CUDA if the synchronization or the copy fails.
+ * Source: none on the pages (error reporting of the allocation-free variant). */
+awq_status awq_get_status_no_alloc(void* stream);
+
 /* Number of kernels awq_linear launches for these sizes on the current device
  * (1, or 2 when the decode GEMV runs its split-row fixup kernel or the GEMM
- * its stream-K fixup kernel; 0 for M == 0 or invalid sizes). Host only. For launch accounting and graph planning;
- * the pages have no counterpart. */
+ * its stream-K fixup kernel; 0 for M == 0 or invalid sizes). Host only. For
+ * launch accounting and graph planning.
+ * Source: none on the pages. */
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group);
 
 /* Self-test of the kernels' failure detection (the pages have no counterpart):
@@ -244,14 +286,17 @@ int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group);
  * GEMM and GEMV pipelines use, on a barrier phase that nothing completes,
  * giving up after `limit_us` microseconds (1 .. 1000000). The expired wait
  * records AWQ_ERR_TIMEOUT in the workspace status word, which awq_get_status
- * then returns; the CUDA context stays usable. Returns AWQ_OK when launched. */
+ * then returns; the CUDA context stays usable. Returns AWQ_OK when launched.
+ * Source: none on the pages (failure detection of this library). */
 awq_status awq_check_bounded_wait(void* workspace, size_t ws_bytes, uint32_t limit_us, void* stream);
 
 /* Synchronize `stream`, then return and clear the device-side status word of
- * `workspace` (AWQ_OK if no device-side error was recorded). */
+ * `workspace` (AWQ_OK if no device-side error was recorded).
+ * Source: none on the pages (error reporting of this library). */
 awq_status awq_get_status(void* workspace, void* stream);
 
-/* Static, human-readable name of a status code. */
+/* Static, human-readable name of a status code.
+ * Source: none on the pages. */
 const char* awq_status_string(awq_status status);
 
 #ifdef __cplusplus

@@ -33,6 +33,19 @@ def test_header_and_binding_agree():
     assert declared_functions() == sorted(awq.EXPORTS)
 
 
+def test_every_declaration_names_its_source():
+    # each entry point's comment ends with "Source:" and the page section that
+    # defines the operation, or says that the pages have none
+    text = open(HEADER).read()
+    for name in declared_functions():
+        m = re.search(r"/\*((?:(?!\*/).)*)\*/\s*(?:awq_status|size_t|int|const char\*)\s+" + name + r"\(", text, re.S)
+        assert m, f"{name}: no comment right before the declaration"
+        src = m.group(1).split("Source:")
+        assert len(src) == 2, f"{name}: no Source line"
+        assert ("TinyChat README" in src[1] or "TensorRT-LLM news item" in src[1]
+                or "none on the pages" in src[1]), name
+
+
 def test_library_exports_every_declared_symbol():
     for name in declared_functions():
         assert hasattr(L, name), name
@@ -191,3 +204,15 @@ def test_fp8_entry_points_reject_bad_arguments():
     bad[6] = FAKE                                    # y on top of x8
     assert L.awq_w4a8_gemm(*bad, 8, 128, 16, 128, FAKE6 + (1 << 24), 256, None) == awq.AWQ_ERR_INVALID_ARG
     assert L.awq_w4a8_gemm(*args, 0, 128, 16, 128, FAKE6 + (1 << 24), 256, None) == awq.AWQ_OK  # empty batch
+
+
+def test_linear_dispatch_follows_the_measured_split():
+    # GEMV up to M = 16 on every layer; from M = 17 to 32 the GEMM on layers
+    # with at least as many 128-channel tiles as SMs (148 here), the GEMV on
+    # narrower ones. The GEMV's split-row plans launch its fixup kernel too;
+    # the GEMM at M <= 32 is data-parallel (one kernel).
+    assert awq.awq_linear_gemv_limit() == 16
+    assert awq.awq_linear_launches(16, 4096, 28672) == 2   # GEMV + fixup
+    assert awq.awq_linear_launches(24, 4096, 28672) == 1   # GEMM: 224 tiles >= 148 SMs
+    assert awq.awq_linear_launches(24, 4096, 4096) == 2    # GEMV + fixup: 32 tiles
+    assert awq.awq_linear_launches(32, 8192, 57344) == 1   # GEMM

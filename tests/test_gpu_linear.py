@@ -386,3 +386,42 @@ def test_decode_m1_one_hot_wide_layer_gives_the_dequantized_weight_exactly():
         x[0, k] = 1.0
         y = _run(awq.awq_w4a16_gemv, x, dev, N)
         assert (y[0].view(np.uint16) == wh[:, k].view(np.uint16)).all(), k
+
+
+# ---- decode at M <= 2: large K and odd row-block counts ----------------------
+# K = 28672 at M = 1 and 2 (224 k-blocks per row); N/16 = 149 row blocks on
+# 148 SMs; N/16 = 1041 (CTA ranges straddling groups, a last group of one row
+# block); K = 14336 at M = 2. Every output against the oracle, and two calls
+# bit for bit equal.
+DECODE_ODD_CASES = [(28672, 512, 1), (28672, 256, 2), (1024, 2384, 1), (1024, 2384, 2), (256, 16656, 1),
+                    (256, 16656, 2), (14336, 1040, 2)]
+
+
+@pytest.mark.parametrize("K,N,M", DECODE_ODD_CASES)
+def test_decode_odd_shapes_match_oracle(K, N, M):
+    W, dev, hp = _packed(N, K, f"rowsk{K}x{N}")
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"rowsk{K}x{N}/x{M}"), M, K, 1.0)
+    y = _run(awq.awq_w4a16_gemv, x, dev, N)
+    y_ref, b = oracle.linear(x, *hp, N, K)
+    check_close(y, y_ref, b, f"decode K={K} N={N} M={M}")
+    y2 = _run(awq.awq_w4a16_gemv, x, dev, N)
+    assert (y2.view(np.uint16) == y.view(np.uint16)).all()        # deterministic
+
+
+# ---- the GEMM at small M on layers with more 128-channel tiles than SMs ----
+# (some CTAs then walk two tiles: the regime where the dequant groups'
+# alternating use of the code stages raced before the previous-phase wait).
+# Against the oracle, and repeated calls bit for bit equal.
+SMALL_M_MANY_TILES = [(4, 1024, 25600, 128), (4, 4096, 28672, 128), (32, 2048, 38400, 128), (16, 1024, 25600, 64)]
+
+
+@pytest.mark.parametrize("M,K,N,group", SMALL_M_MANY_TILES)
+def test_gemm_small_m_many_tiles(M, K, N, group):
+    W, dev, hp = _packed(N, K, f"smt{K}x{N}", group=group)
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"smt{K}x{N}/x{M}"), M, K, 1.0)
+    ys = [_run(awq.awq_w4a16_gemm, x, dev, N, group=group) for _ in range(5)]
+    for y in ys[1:]:
+        assert (y.view(np.uint16) == ys[0].view(np.uint16)).all()
+    rows = sample_rows(N, 256, seed=M)
+    y_ref, b = oracle_rows(x, *hp, N, K, rows, group)
+    check_close(ys[0][:, rows], y_ref, b, f"gemm M={M} K={K} N={N} group={group}")

@@ -2,12 +2,15 @@
 device memory (e.g. code confined to a fixed memory pool, or a plug-in whose
 host process owns every device allocation).
 
-It is called here through the C ABI (ctypes) and compared, on two calls in a
-row, with the workspace entry point awq_w4a16_gemv, within the tolerance of
-the other parity tests (|a - b| <= 2e-3 * sum|x w| + 1e-3). Sizes whose
-scratch would exceed AWQ_GEMV_NO_ALLOC_SCRATCH_BYTES must be rejected with
-AWQ_ERR_WORKSPACE before anything runs. This file is collected last so that a
-run stopping at the first failure has run every other test before it.
+It is called here through the C ABI (ctypes) on two calls in a row and must
+give the same y, bit for bit, as the workspace entry point awq_w4a16_gemv (the
+same kernels run in the same order), and y within the tolerance of the other
+parity tests of the fp64 oracle (|y - y_ref| <= 2e-3 * sum|x w| + 1e-3). Its
+status word, read back with awq_get_status_no_alloc, must stay AWQ_OK. Sizes
+whose scratch would exceed AWQ_GEMV_NO_ALLOC_SCRATCH_BYTES must be rejected
+with AWQ_ERR_WORKSPACE, and a y that overlaps an input with
+AWQ_ERR_INVALID_ARG, before anything runs. This file is collected last so that
+a run stopping at the first failure has run every other test before it.
 """
 import numpy as np
 import pytest
@@ -16,7 +19,7 @@ import torch
 import awq_synth
 import oracle
 import weight_only_bit_awq_b200 as awq
-from gpu_helpers import ABS_TOL, REL_TOL, gpu_pack, host, packed_to_host, to_dev
+from gpu_helpers import check_close, gpu_pack, host, packed_to_host, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -48,17 +51,16 @@ def test_matches_the_workspace_entry_point_on_two_calls_in_a_row(K, N, M):
         assert (y == 0).all()          # rejected before anything ran
         return
     ws = awq.new_workspace(M, K, N, xd.device)
-    y_ws = host(awq.awq_w4a16_gemv(xd, *dev, N, ws), np.float16).astype(np.float64)
-    q, z, s = oracle.unpack(*hp, N, K)
-    wh = oracle.dequant(q, z, s).astype(np.float64)
-    bound = np.abs(x.astype(np.float64)) @ np.abs(wh).T
+    y_ws = host(awq.awq_w4a16_gemv(xd, *dev, N, ws), np.uint16)
+    assert awq.awq_get_status(ws) == awq.AWQ_OK
+    y_ref, bound = oracle.linear(x, *hp, N, K)
     for call in range(2):
         y.fill_(float("nan"))
         assert _no_alloc(xd, *dev, y, N) == awq.AWQ_OK
-        torch.cuda.synchronize()
-        y_na = host(y, np.float16).astype(np.float64)
-        err = np.abs(y_na - y_ws)
-        assert (err <= REL_TOL * bound + ABS_TOL).all(), (call, float(err.max()))
+        assert awq.awq_get_status_no_alloc() == awq.AWQ_OK
+        y_na = host(y, np.uint16)
+        assert np.array_equal(y_na, y_ws), (call, int((y_na != y_ws).sum()))
+        check_close(y_na.view(np.float16), y_ref, bound, f"no-alloc call {call}, M={M} K={K} N={N}")
 
 
 def test_sizes_beyond_the_scratch_are_rejected():
@@ -89,3 +91,8 @@ def test_argument_errors():
     assert L.awq_w4a16_gemv_no_alloc(*args, 1, 128, 16, 96, s) == awq.AWQ_ERR_UNSUPPORTED
     assert L.awq_w4a16_gemv_no_alloc(None, *args[1:], 1, 128, 16, 128, s) == awq.AWQ_ERR_INVALID_ARG
     assert L.awq_w4a16_gemv_no_alloc(*args, 0, 128, 16, 128, s) == awq.AWQ_OK
+    # y overlapping x, the codes, the scales or the zeros
+    for alias in (x, qw, sc, ze):
+        bad = [x.data_ptr(), qw.data_ptr(), sc.data_ptr(), ze.data_ptr(), alias.data_ptr()]
+        assert L.awq_w4a16_gemv_no_alloc(*bad, 1, 128, 16, 128, s) == awq.AWQ_ERR_INVALID_ARG
+    assert awq.awq_get_status_no_alloc() == awq.AWQ_OK

@@ -10,7 +10,8 @@ Functions (same names as the C entry points):
   awq_packed_size, awq_workspace_bytes, awq_workspace_init, awq_pack,
   awq_dequant, awq_w4a16_gemv, awq_w4a16_gemm, awq_linear,
   awq_linear_gemv_limit, awq_linear_launches, awq_check_bounded_wait,
-  awq_get_status, awq_status_string, awq_w4a16_gemv_no_alloc, and the W4A8-FP8
+  awq_get_status, awq_status_string, awq_w4a16_gemv_no_alloc,
+  awq_get_status_no_alloc, and the W4A8-FP8
   variant awq_fp8_row_exponents, awq_fp8_quantize_x, awq_dequant_fp8,
   awq_w4a8_gemm.
 """
@@ -22,21 +23,25 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libawq_b200.so")
+# AWQ_B200_DEBUG=1 loads the debug build (every guarded device access checks
+# its index range and records AWQ_ERR_BOUNDS instead of faulting).
+DEBUG = os.environ.get("AWQ_B200_DEBUG", "") == "1"
+LIB_PATH = os.path.join(_PKG, "libawq_b200_debug.so" if DEBUG else "libawq_b200.so")
 
 GROUP = 128
 GEMV_MAX_M = 32
 
 STATUS_NAMES = {
     0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_SHAPE", 3: "AWQ_ERR_ALIGNMENT", 4: "AWQ_ERR_WORKSPACE",
-    5: "AWQ_ERR_UNSUPPORTED", 6: "AWQ_ERR_CUDA", 7: "AWQ_ERR_TIMEOUT", 8: "AWQ_ERR_NONFINITE",
+    5: "AWQ_ERR_UNSUPPORTED", 6: "AWQ_ERR_CUDA", 7: "AWQ_ERR_TIMEOUT", 8: "AWQ_ERR_NONFINITE", 9: "AWQ_ERR_BOUNDS",
 }
 globals().update({name: code for code, name in STATUS_NAMES.items()})
 
 # Every symbol include/awq.h declares.
 EXPORTS = ("awq_packed_size", "awq_workspace_bytes", "awq_workspace_init", "awq_pack", "awq_dequant",
            "awq_w4a16_gemv", "awq_w4a16_gemm", "awq_linear", "awq_linear_gemv_limit", "awq_get_status",
-           "awq_status_string", "awq_w4a16_gemv_no_alloc", "awq_linear_launches", "awq_check_bounded_wait",
+           "awq_status_string", "awq_w4a16_gemv_no_alloc", "awq_get_status_no_alloc", "awq_linear_launches",
+           "awq_check_bounded_wait",
            "awq_fp8_row_exponents", "awq_fp8_quantize_x", "awq_dequant_fp8", "awq_w4a8_gemm")
 
 
@@ -63,7 +68,7 @@ def _build_module():
 def _load() -> ctypes.CDLL:
     # (Re)compile in-tree with nvcc when the library is missing or older than
     # its sources; a failed build raises, there is no fallback.
-    _build_module().build()
+    _build_module().build(debug=DEBUG)
     lib = ctypes.CDLL(LIB_PATH)
     vp, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     lib.awq_packed_size.argtypes = [i64, i64, ci, ctypes.POINTER(_PackedSizes)]
@@ -75,6 +80,7 @@ def _load() -> ctypes.CDLL:
     for f in ("awq_w4a16_gemv", "awq_w4a16_gemm", "awq_linear"):
         getattr(lib, f).argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, sz, vp]
     lib.awq_w4a16_gemv_no_alloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp]
+    lib.awq_get_status_no_alloc.argtypes = [vp]
     lib.awq_linear_gemv_limit.argtypes = []
     lib.awq_linear_launches.argtypes = [i64, i64, i64, ci]
     lib.awq_check_bounded_wait.argtypes = [vp, sz, ctypes.c_uint32, vp]
@@ -188,7 +194,8 @@ def awq_w4a16_gemm(x, qweight, scales, zeros, N, workspace, group: int = GROUP, 
 
 
 def awq_linear(x, qweight, scales, zeros, N, workspace, group: int = GROUP, y=None):
-    """The linear layer: GEMV for M <= awq_linear_gemv_limit(), GEMM above."""
+    """The linear layer: the GEMV for M <= awq_linear_gemv_limit() (and up to
+    M = 32 on layers with fewer 128-channel tiles than SMs), the GEMM otherwise."""
     return _linear_call(lib.awq_linear, "awq_linear", x, qweight, scales, zeros, N, workspace, group, y)
 
 
@@ -204,6 +211,12 @@ def awq_w4a16_gemv_no_alloc(x, qweight, scales, zeros, N, group: int = GROUP, y=
                                        _dev(y, torch.float16, "y"), M, K, N, group, _stream(x)),
            "awq_w4a16_gemv_no_alloc")
     return y
+
+
+def awq_get_status_no_alloc(device=None) -> int:
+    """Synchronize the current stream; return (and clear) the status word of
+    the no-alloc GEMV's scratch array on the current device."""
+    return int(lib.awq_get_status_no_alloc(torch.cuda.current_stream(device).cuda_stream))
 
 
 def awq_fp8_row_exponents(scales: torch.Tensor, K: int, N: int, group: int = GROUP) -> torch.Tensor:

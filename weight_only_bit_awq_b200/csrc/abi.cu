@@ -136,7 +136,18 @@ awq_status gemm_impl(const LinearArgs& a, cudaStream_t stream) {
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
-int g_gemv_limit = AWQ_GEMV_MAX_M;
+// Dispatch of awq_linear between the decode GEMV and the tensor-core GEMM,
+// from measurements on B200 (CUDA graphs, rotating weights, LLaMA-3-8B and
+// LLaMA-2-70B decode layers at M = 4 .. 64): the GEMV is faster on every layer
+// up to M = 16; at M = 24 and 32 the GEMM is faster on layers with at least
+// as many 128-channel tiles as SMs (gate_up: 54.6 against 76.4 us at M = 32
+// on LLaMA-3-8B, 195.6 against 256.3 us on 70B) and slower on the narrower
+// ones, which leave most SMs without a tile.
+constexpr int kGemvAlwaysM = 16;
+
+bool linear_uses_gemv(int64_t M, int64_t N, int sm_count) {
+  return M <= kGemvAlwaysM || (M <= AWQ_GEMV_MAX_M && (N + 127) / 128 < sm_count);
+}
 
 }  // namespace
 
@@ -239,11 +250,11 @@ awq_status awq_linear(const void* x, const void* qweight, const void* scales, co
   if (st != AWQ_OK) return st;
   if (M == 0) return AWQ_OK;
   if ((st = check_device()) != AWQ_OK) return st;
-  if (M <= g_gemv_limit) return gemv_impl(a, static_cast<cudaStream_t>(stream));
+  if (linear_uses_gemv(M, N, device_info().sm_count)) return gemv_impl(a, static_cast<cudaStream_t>(stream));
   return gemm_impl(a, static_cast<cudaStream_t>(stream));
 }
 
-int awq_linear_gemv_limit(void) { return g_gemv_limit; }
+int awq_linear_gemv_limit(void) { return kGemvAlwaysM; }
 
 awq_status awq_fp8_row_exponents(const void* scales, int64_t K, int64_t N, int group, void* e_out, void* stream) {
   awq_status st = check_kn(K, N, group);
@@ -321,8 +332,9 @@ awq_status awq_w4a8_gemm(const void* x8, const void* sx, const void* qweight, co
 
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group) {
   if (M <= 0 || M > kMaxM || check_kn(K, N, group) != AWQ_OK) return 0;
-  if (M > g_gemv_limit) return plan_gemm(M, K, N, sm_count_or_default()).stream_k ? 2 : 1;
-  return plan_gemv(M, K, N, group, sm_count_or_default()).has_split ? 2 : 1;
+  const int sms = sm_count_or_default();
+  if (!linear_uses_gemv(M, N, sms)) return plan_gemm(M, K, N, sms).stream_k ? 2 : 1;
+  return plan_gemv(M, K, N, group, sms).has_split ? 2 : 1;
 }
 
 awq_status awq_check_bounded_wait(void* workspace, size_t ws_bytes, uint32_t limit_us, void* stream) {
@@ -357,6 +369,7 @@ const char* awq_status_string(awq_status status) {
     case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: a CUDA call or kernel launch failed";
     case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT: a bounded wait on the device expired";
     case AWQ_ERR_NONFINITE: return "AWQ_ERR_NONFINITE: awq_pack met an inf or NaN weight";
+    case AWQ_ERR_BOUNDS: return "AWQ_ERR_BOUNDS: a device-side index check of the debug build failed";
   }
   return "unknown awq_status";
 }

@@ -49,6 +49,31 @@ __device__ __forceinline__ void record_status(uint32_t* status, uint32_t code) {
   if (status) atomicCAS(status, 0u, code);
 }
 
+// Bounds checks of the debug build (compiled with -DAWQ_DEBUG; build.py
+// --debug writes libawq_b200_debug.so). A guarded global or shared access
+// first checks that its whole range lies inside its buffer; a failed check
+// records AWQ_ERR_BOUNDS in the status word and the access is skipped, so the
+// kernel neither faults nor traps. In the normal build the checks are `true`
+// and compile to nothing.
+__host__ __device__ __forceinline__ constexpr bool in_range(int64_t off, int64_t len, int64_t size) {
+  return off >= 0 && len >= 0 && off + len <= size;
+}
+#ifdef AWQ_DEBUG
+__device__ __forceinline__ bool debug_check(bool ok, uint32_t* status) {
+  if (!ok) record_status(status, AWQ_ERR_BOUNDS);
+  return ok;
+}
+// Bytes of dynamic shared memory this CTA was launched with.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t r;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+#define AWQ_CHECK(cond, status) ::awq::debug_check((cond), (status))
+#else
+#define AWQ_CHECK(cond, status) true
+#endif
+
 // Per-device facts gathered once.
 struct DeviceInfo {
   int device = -1;
@@ -63,10 +88,10 @@ struct GemvPlan {
   int group;            // quantization group size (128, 64 or 32)
   int nt;               // token tiles of 8 (1, 2 or 4)
   bool int_path;        // M <= 2, groups of 128: integer MMAs on the codes and x digits
-  int ku;               // k-blocks per streamed unit (1, 2 or 4)
+  int ku;               // k-blocks per streamed unit
   int stages;           // depth of the shared-memory ring
   size_t smem_bytes;    // dynamic shared memory per CTA
-  int ctas;             // persistent CTAs (up to two per SM)
+  int ctas;             // persistent CTAs
   int groups;           // groups of 8 row blocks
   bool has_split;       // some group is split between CTAs (the fixup kernel runs)
   size_t partial_off;   // workspace offset of the split-row partial sums (bytes)

@@ -27,6 +27,7 @@
 // the epilogue of one tile while the next is accumulated. Every
 // mbarrier wait is bounded; on expiry AWQ_ERR_TIMEOUT goes to the status word
 // and the CTA drains and exits.
+#include <atomic>
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
@@ -529,14 +530,14 @@ cudaError_t launch_bn(const uint8_t* x8, const float* sx, const uint32_t* qweigh
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  static uint64_t attr_set = 0;  // one bit per device that has the attribute
+  static std::atomic<uint64_t> attr_set{0};  // one bit per device that has the attribute
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
-  if (!(attr_set >> dev & 1)) {
+  if (!(attr_set.load(std::memory_order_acquire) >> dev & 1)) {
     cudaError_t e =
         cudaFuncSetAttribute(gemm_fp8_kernel<BN, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
-    attr_set |= uint64_t(1) << dev;
+    attr_set.fetch_or(uint64_t(1) << dev, std::memory_order_acq_rel);
   }
   const int64_t tiles = ((M + BN - 1) / BN) * ((N + kBM - 1) / kBM);
   const int ctas = (int)(tiles < device_info().sm_count ? tiles : device_info().sm_count);  // one per SM

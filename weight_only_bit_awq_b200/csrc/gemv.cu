@@ -45,10 +45,12 @@
 // plain stores, so streaming never waits on another CTA; a small fixup
 // kernel launched right behind the GEMV (programmatic dependent launch) adds
 // the slots in CTA order (deterministic) and writes y.
+#include <atomic>
 #include <type_traits>
 
 #include "awq_internal.cuh"
 #include "sm100_ptx.cuh"
+#include "gemv_common.cuh"
 
 namespace awq {
 namespace {
@@ -56,23 +58,11 @@ namespace {
 constexpr int kConsumers = kGroupBlocks;  // one consumer warp per row block of a unit
 constexpr int kWarpXsum = 1 + kConsumers;  // per-k-block sums of x (M <= 8)
 constexpr int kThreads = (2 + kConsumers) * 32;
-constexpr int kMaxStages = 16;
-constexpr int kKbQBytes = kGroupBlocks * 1024;                    // codes of one k-block of a group
-constexpr int kKbScaleBytes = kGroupBlocks * kRowsPerBlock * 2;   // 256: one row of scales (one group)
-constexpr int kKbZeroBytes = kGroupBlocks * kRowsPerBlock / 2;    // 64: one row of zero points
-constexpr int kKbXsBytes = 8 * 2 * 4;                             // 8 tokens x (C, X) fp32, per group
-constexpr int kXRowBytes = kKPerBlock * 2;                        // 256 bytes of x per token and k-block
 // Shared memory one CTA may use (two CTAs per SM share 228 KiB, minus the
 // 1 KiB per CTA the hardware reserves).
 constexpr int kSmemPerCta2 = 112 * 1024;
 constexpr int kSmemPerCta1 = 226 * 1024;
 
-// Integer path (M <= 2, groups of 128): per k-block, the x-prep warp writes
-// the B fragments of the integer MMAs -- for each lane column t (0..3), 4 M
-// digit columns of 32 bytes, plus one 32-byte pad per t so that its stores are
-// bank-conflict free -- and one float4 of coefficients per t.
-__host__ __device__ constexpr int int_bfrag_tstride(int M) { return (4 * M + 1) * 32; }
-__host__ __device__ constexpr int int_xs_bytes(int M) { return 4 * int_bfrag_tstride(M) + 64; }
 
 // Byte offsets inside one ring stage for a unit of up to KU k-blocks, M
 // tokens and groups of GS inputs (the same numbers on the host and in every
@@ -90,165 +80,6 @@ struct Stage {
     bytes = x + M * KU * kXRowBytes;  // every term is a multiple of 16
   }
 };
-
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));  // (a & b) | c
-  return d;
-}
-__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
-__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
-
-// d += A B (m16n8k16, fp16 inputs, fp32 accumulate).
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-// d = A B (the accumulator input is zero; no separate clearing of d).
-__device__ __forceinline__ void mma_16816_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                                uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%10,%10,%10,%10};"
-      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
-}
-
-// d += A B (m16n8k32, A unsigned bytes, B signed bytes, exact s32 accumulate);
-// the _first form starts from zero.
-__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                           uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void imma_16832_first(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                                 uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%10,%10,%10,%10};"
-      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
-}
-
-// Group size GS (128, 64 or 32) in the k-block of 128: the packed layout puts
-// the inputs of group j / J (J = GS / 32) into word 4t + j of every lane t, so
-// the MMAs of step j (one word per lane) see a single group. kGroupsPerKb
-// groups per k-block, each with its own scale and zero point.
-template <int GS>
-struct Grp {
-  static constexpr int J = GS / 32;              // MMA steps j per group
-  static constexpr int kPerKb = kKPerBlock / GS;  // groups per k-block
-  // byte offset, in a token's 128 x values of the k-block, of the 8 inputs in word 4t + j
-  __host__ __device__ static constexpr int x_off(int t, int j) { return 2 * word_k0(4 * t + j, GS); }
-};
-
-// Accumulators per token tile (M > 8): for GS = 128 the 8 MMAs of a k-block
-// are spread over two chains so that consecutive MMAs do not wait on each
-// other; for smaller groups there is one accumulator per group.
-template <int NT, int GS>
-struct Chains {
-  static constexpr int value = GS == 128 ? 2 : Grp<GS>::kPerKb;
-};
-
-// acc[c][nt] = (q - z) * x over one k-block, rows g and g+8 (M > 8); za, zb
-// are the zero points of the rows per group of the k-block.
-template <int NT, int GS>
-__device__ __forceinline__ void block_mma(float (&acc)[Chains<NT, GS>::value][NT][4], const uint4& wa4,
-                                          const uint4& wb4, const uint32_t (&za)[Grp<GS>::kPerKb],
-                                          const uint32_t (&zb)[Grp<GS>::kPerKb], const uint4 (&xf)[NT][4]) {
-  constexpr int C = Chains<NT, GS>::value, J = Grp<GS>::J;
-  const uint32_t kMaskLo = 0x000F000Fu, kMaskHi = 0x00F000F0u, kMagic = 0x64006400u;
-  const __half2 sixteenth = u32_as_h2(0x2C002C00u);  // 1/16
-  const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
-  const uint32_t wb[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    // Constants built from bit patterns (integer ops only, no conversions):
-    // fp16 1024 + z is 0x6400 + z, and -(64 + z) is 0xD400 + 16 z (z <= 15).
-    const int gk = j / J;
-    const __half2 zlo_a = u32_as_h2((0x6400u + za[gk]) * 0x00010001u);
-    const __half2 zlo_b = u32_as_h2((0x6400u + zb[gk]) * 0x00010001u);
-    const __half2 zhi_a = u32_as_h2((0xD400u + (za[gk] << 4)) * 0x00010001u);
-    const __half2 zhi_b = u32_as_h2((0xD400u + (zb[gk] << 4)) * 0x00010001u);
-    uint32_t a = wa[j], b = wb[j];
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const uint32_t a0 = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(a, kMaskLo, kMagic)), zlo_a));
-      const uint32_t a1 = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(b, kMaskLo, kMagic)), zlo_b));
-      const uint32_t a2 = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(a, kMaskHi, kMagic)), sixteenth, zhi_a));
-      const uint32_t a3 = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(b, kMaskHi, kMagic)), sixteenth, zhi_b));
-      const int step = 2 * j + half;
-      const int idx = GS == 128 ? step % C : gk;
-      const bool first = GS == 128 ? step < C : (j % J == 0 && half == 0);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint32_t b0 = half ? xf[nt][j].z : xf[nt][j].x;
-        const uint32_t b1 = half ? xf[nt][j].w : xf[nt][j].y;
-        if (first)
-          mma_16816_first(acc[idx][nt], a0, a1, a2, a3, b0, b1);
-        else
-          mma_16816(acc[idx][nt], a0, a1, a2, a3, b0, b1);
-      }
-      a >>= 8;
-      b >>= 8;
-    }
-  }
-}
-
-// fp16 bits -> fp32 value of a non-negative fp16 (scales), exact for normal and
-// subnormal inputs: the 15 value bits shifted into place read as fp32 are the
-// value times 2^-112.
-__device__ __forceinline__ float pos_half_bits_to_float(uint32_t h) {
-  return __uint_as_float(h << 13) * 5.192296858534828e+33f;  // 2^112; the sign bit of h is 0
-}
-
-// M <= 8 (one token tile): the codes go into the MMA unchanged, as the fp16
-// values 1024 + q (pairs taken with the 0x000F000F mask, "lo" k) and
-// 1024 + 16 q (0x00F000F0 mask, "hi" k), in separate MMAs so that the two
-// offsets can be removed afterwards with per-group sums of x:
-//   sum_k x (q - z) = acc_lo + acc_hi / 16 - (1024 X_lo + 64 X_hi) - z (X_lo + X_hi)
-// with X_lo, X_hi the sums of x over the lo and hi k of the group. This needs
-// 5 integer ops per 8 weights and no fp16 arithmetic. LoHi<GS>::kAcc
-// accumulators: lo ones first, then hi ones; for GS = 128 two chains of each,
-// else one of each per group.
-template <int GS>
-struct LoHi {
-  static constexpr int kLo = GS == 128 ? 2 : Grp<GS>::kPerKb;
-  static constexpr int kAcc = 2 * kLo;
-};
-template <int GS>
-__device__ __forceinline__ void block_mma_lohi(float (&acc)[LoHi<GS>::kAcc][4], const uint4& wa4, const uint4& wb4,
-                                               const uint4 (&xf)[4]) {
-  constexpr int kLo = LoHi<GS>::kLo, J = Grp<GS>::J;
-  const uint32_t kMaskLo = 0x000F000Fu, kMaskHi = 0x00F000F0u, kMagic = 0x64006400u;
-  const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
-  const uint32_t wb[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t a = wa[j], b = wb[j], a8 = wa[j] >> 8, b8 = wb[j] >> 8;
-    // slots (2t, 2t+1) <- k0 + 0, 1 (lo) / 2, 3 (hi); slots (2t+8, 2t+9) <- k0 + 4, 5 / 6, 7
-    const uint32_t l0 = lop3_and_or(a, kMaskLo, kMagic), l1 = lop3_and_or(b, kMaskLo, kMagic);
-    const uint32_t l2 = lop3_and_or(a8, kMaskLo, kMagic), l3 = lop3_and_or(b8, kMaskLo, kMagic);
-    const uint32_t h0 = lop3_and_or(a, kMaskHi, kMagic), h1 = lop3_and_or(b, kMaskHi, kMagic);
-    const uint32_t h2 = lop3_and_or(a8, kMaskHi, kMagic), h3 = lop3_and_or(b8, kMaskHi, kMagic);
-    const int idx = GS == 128 ? (j & 1) : j / J;
-    const bool first = GS == 128 ? j < 2 : j % J == 0;
-    if (first) {
-      mma_16816_first(acc[idx], l0, l1, l2, l3, xf[j].x, xf[j].z);
-      mma_16816_first(acc[kLo + idx], h0, h1, h2, h3, xf[j].y, xf[j].w);
-    } else {
-      mma_16816(acc[idx], l0, l1, l2, l3, xf[j].x, xf[j].z);
-      mma_16816(acc[kLo + idx], h0, h1, h2, h3, xf[j].y, xf[j].w);
-    }
-  }
-}
 
 // M <= 2, groups of 128 ("integer path"): exact integer MMAs on the codes.
 // Per k-block and token, the x-prep warp writes x as a block fixed-point
@@ -292,7 +123,7 @@ template <int NT, int KU, bool kM1, int GS, bool kInt>
 __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
     gemv_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight, const __half* __restrict__ scales,
                 const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M, int K, int N, int NS,
-                float* __restrict__ partial, uint32_t* status) {
+                float* __restrict__ partial, int64_t part_floats, uint32_t* status) {
   extern __shared__ __align__(16) uint8_t smem[];
   static_assert(!kInt || (NT == 1 && GS == 128 && !kM1), "integer path: one token tile, groups of 128");
   constexpr bool kLoHi = NT == 1 && !kInt;
@@ -336,21 +167,34 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       const int64_t kb0 = (int64_t)cj * KU;
       const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
       const uint32_t st = sbase + s * L.bytes;
+      const int64_t qw0 = unit_first_block(cgi, kb0, rg.KB, rg.NB) * kWordsPerBlock;
+      const bool qok = AWQ_CHECK(in_range(qw0, (int64_t)ku * R * 256, (int64_t)K * N / 8) &&
+                                     in_range(s * L.bytes + L.q, ku * R * 1024, dynamic_smem_bytes()),
+                                 status);
       if (lane == 0)
-        ptx::mbar_arrive_expect_tx(full(s), (uint32_t)(ku * R * 1024 + (kXWarp ? 0 : M * ku * kXRowBytes)));
+        ptx::mbar_arrive_expect_tx(full(s),
+                                   (uint32_t)((qok ? ku * R * 1024 : 0) + (kXWarp ? 0 : M * ku * kXRowBytes)));
       __syncwarp();
-      if (lane == 0)
-        ptx::bulk_g2s(st + L.q, qweight + unit_first_block(cgi, kb0, rg.KB, rg.NB) * kWordsPerBlock,
-                      (uint32_t)(ku * R * 1024), full(s));
+      if (lane == 0 && qok) ptx::bulk_g2s(st + L.q, qweight + qw0, (uint32_t)(ku * R * 1024), full(s));
       const __half* srow = scales + kb0 * kGPK * N + kGroupBlocks * kRowsPerBlock * cgi;
       for (int p = lane; p < ku * kGPK * 16; p += 32) {  // ku * kGPK rows of 32 R bytes
         const int j = p >> 4, l = p & 15;
-        if (l < 2 * R) ptx::cp_async_16(st + L.s + j * kKbScaleBytes + 16 * l, srow + (int64_t)j * N + 8 * l);
+        if (l < 2 * R &&
+            AWQ_CHECK(in_range(kb0 * kGPK * N + kGroupBlocks * kRowsPerBlock * cgi + (int64_t)j * N + 8 * l, 8,
+                               (int64_t)(K / GS) * N) &&
+                          in_range(s * L.bytes + L.s + j * kKbScaleBytes + 16 * l, 16, dynamic_smem_bytes()),
+                      status))
+          ptx::cp_async_16(st + L.s + j * kKbScaleBytes + 16 * l, srow + (int64_t)j * N + 8 * l);
       }
       const uint8_t* zrow = zeros + kb0 * kGPK * (N / 2) + 64 * cgi;
       for (int p = lane; p < ku * kGPK * 8; p += 32) {  // ku * kGPK rows of 8 R bytes
         const int j = p >> 3, l = p & 7;
-        if (l < R) ptx::cp_async_8(st + L.z + j * kKbZeroBytes + 8 * l, zrow + (int64_t)j * (N / 2) + 8 * l);
+        if (l < R &&
+            AWQ_CHECK(in_range(kb0 * kGPK * (N / 2) + 64 * cgi + (int64_t)j * (N / 2) + 8 * l, 8,
+                               (int64_t)(K / GS) * (N / 2)) &&
+                          in_range(s * L.bytes + L.z + j * kKbZeroBytes + 8 * l, 8, dynamic_smem_bytes()),
+                      status))
+          ptx::cp_async_8(st + L.z + j * kKbZeroBytes + 8 * l, zrow + (int64_t)j * (N / 2) + 8 * l);
       }
       ptx::cp_async_arrive_noinc(full(s));
       if (++cj == rg.UPG) {
@@ -367,9 +211,19 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
         if (lane == 0) ptx::mbar_arrive_expect_tx(xb, (uint32_t)(M * ku * kXRowBytes));
         __syncwarp();
       }
-      if (lane < M)
-        ptx::bulk_g2s(sbase + s * L.bytes + L.x + KU * kXRowBytes * lane, x + (int64_t)lane * K + kb0 * kKPerBlock,
-                      (uint32_t)(ku * kXRowBytes), xb);
+      if (lane < M) {
+        // a copy that fails its check is replaced by an arrival with its byte count
+        if (AWQ_CHECK(in_range((int64_t)lane * K + kb0 * kKPerBlock, (int64_t)ku * kKPerBlock, (int64_t)M * K) &&
+                          in_range(s * L.bytes + L.x + KU * kXRowBytes * lane, ku * kXRowBytes, dynamic_smem_bytes()),
+                      status))
+          ptx::bulk_g2s(sbase + s * L.bytes + L.x + KU * kXRowBytes * lane, x + (int64_t)lane * K + kb0 * kKPerBlock,
+                        (uint32_t)(ku * kXRowBytes), xb);
+#ifdef AWQ_DEBUG
+        else
+          asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(xb), "r"((uint32_t)(ku * kXRowBytes))
+                       : "memory");
+#endif
+      }
       if (++xj == rg.UPG) xj = 0;
     };
     const int pro = n_units < NS ? n_units : NS;
@@ -550,7 +404,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int m = 8 * nt + 2 * t + (cc & 1);
-        if (m < M) y[(int64_t)m * N + ra + 8 * (cc >> 1)] = __float2half_rn(v[nt][cc]);
+        if (m < M && AWQ_CHECK(in_range((int64_t)m * N + ra + 8 * (cc >> 1), 1, (int64_t)M * N), status))
+          y[(int64_t)m * N + ra + 8 * (cc >> 1)] = __float2half_rn(v[nt][cc]);
       }
   };
   // Partial slot of CTA `cta` for group g_: [cta][first/last group of cta][row block][16 rows][M].
@@ -566,7 +421,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int m = 8 * nt + 2 * t + (cc & 1);
-        if (m < M) mine[(g + 8 * (cc >> 1)) * M + m] = v[nt][cc];
+        if (m < M && AWQ_CHECK(in_range(mine - partial + (g + 8 * (cc >> 1)) * M + m, 1, part_floats), status))
+          mine[(g + 8 * (cc >> 1)) * M + m] = v[nt][cc];
       }
   };
   // Output of a finished group: fp16 y if this CTA saw all of its k-blocks,
@@ -583,12 +439,16 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       if ((t & 1) || m >= M) return;
       const int64_t ra = (g_ * kGroupBlocks + cw) * kRowsPerBlock + g;
       if (covered(g_)) {
-        y[(int64_t)m * N + ra] = __float2half_rn(r0);
-        y[(int64_t)m * N + ra + 8] = __float2half_rn(r1);
+        if (AWQ_CHECK(in_range((int64_t)m * N + ra, 9, (int64_t)M * N), status)) {
+          y[(int64_t)m * N + ra] = __float2half_rn(r0);
+          y[(int64_t)m * N + ra + 8] = __float2half_rn(r1);
+        }
       } else {
         float* mine = slot(c, g_);
-        mine[g * M + m] = r0;
-        mine[(g + 8) * M + m] = r1;
+        if (AWQ_CHECK(in_range(mine - partial + g * M + m, 8 * M + 1, part_floats), status)) {
+          mine[g * M + m] = r0;
+          mine[(g + 8) * M + m] = r1;
+        }
       }
       return;
     }
@@ -754,7 +614,11 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       const uint8_t* st = smem + s * L.bytes;
       const int64_t kb0 = (int64_t)jj * KU;
       const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
-      if (ku == KU) {
+      if (!AWQ_CHECK(in_range(s * L.bytes + L.q, (ku * R) * 1024, dynamic_smem_bytes()) &&
+                         in_range(s * L.bytes + L.x, M * KU * kXRowBytes, dynamic_smem_bytes()),
+                     status)) {
+        // (debug build) a stage that fails its check is skipped
+      } else if (ku == KU) {
         // no guard: for one token tile pairs of k-blocks can interleave (more
         // token tiles would run out of registers)
         constexpr int kUnroll = NT == 1 ? 2 : 1;
@@ -786,7 +650,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
 // leave free on an SM, so fixup CTAs can be resident and waiting before the
 // GEMV's CTAs exit.)
 __global__ void __launch_bounds__(128, 16) gemv_fixup_kernel(const float* __restrict__ partial, __half* __restrict__ y,
-                                                          int M, int K, int N, int KU, int P) {
+                                                          int M, int K, int N, int KU, int P, int64_t part_floats,
+                                                          uint32_t* status) {
   ptx::griddep_launch_dependents();
   const Range rg(K, N, KU, P);
   const int64_t gi = blockIdx.x;
@@ -801,6 +666,11 @@ __global__ void __launch_bounds__(128, 16) gemv_fixup_kernel(const float* __rest
   const int which_first = rg.first_unit(c_first) == gi * rg.UPG ? 0 : 1;
   const int n = (int)(c_last - c_first);  // contributors after the first
   ptx::griddep_wait();
+  if (!AWQ_CHECK(in_range(p - partial + which_first * slot_floats, 1, part_floats) &&
+                     in_range(p - partial + (int64_t)n * cta_floats, 1, part_floats) &&
+                     in_range((int64_t)m * N + gi * kGroupBlocks * kRowsPerBlock + threadIdx.x, 1, (int64_t)M * N),
+                 status))
+    return;
   float v = __ldcg(p + which_first * slot_floats);
   for (int q0 = 1; q0 <= n; q0 += 4) {
     float part[4];
@@ -815,14 +685,14 @@ __global__ void __launch_bounds__(128, 16) gemv_fixup_kernel(const float* __rest
 template <int NT, int KU, bool kM1, int GS, bool kInt>
 cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros, __half* y,
                      int M, int K, int N, void* workspace, const GemvPlan& p, cudaStream_t stream) {
-  static uint64_t attr_set = 0;  // one bit per device
+  static std::atomic<uint64_t> attr_set{0};  // one bit per device that has the attribute
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
-  if (!(attr_set >> dev & 1)) {
+  if (!(attr_set.load(std::memory_order_acquire) >> dev & 1)) {
     cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, KU, kM1, GS, kInt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          NT == 4 ? kSmemPerCta1 : kSmemPerCta2);
     if (e != cudaSuccess) return e;
-    attr_set |= uint64_t(1) << dev;
+    attr_set.fetch_or(uint64_t(1) << dev, std::memory_order_acq_rel);
   }
   char* ws = static_cast<char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
@@ -837,14 +707,16 @@ cudaError_t launch_t(const __half* x, const uint32_t* qweight, const __half* sca
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const int64_t part_floats = (int64_t)(p.ws_bytes - p.partial_off) / 4;
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<NT, KU, kM1, GS, kInt>, x, qweight, scales, zeros, y, M, K, N,
-                                     p.stages, partial, status);
+                                     p.stages, partial, part_floats, status);
   if (e != cudaSuccess || !p.has_split) return e;
   cudaLaunchConfig_t fcfg = cfg;
   fcfg.gridDim = dim3((unsigned)p.groups, (unsigned)M);
   fcfg.blockDim = dim3(kGroupBlocks * kRowsPerBlock);
   fcfg.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&fcfg, gemv_fixup_kernel, (const float*)partial, y, M, K, N, p.ku, p.ctas);
+  return cudaLaunchKernelEx(&fcfg, gemv_fixup_kernel, (const float*)partial, y, M, K, N, p.ku, p.ctas, part_floats,
+                            status);
 }
 
 template <int NT, bool kM1, int GS, bool kInt = false>

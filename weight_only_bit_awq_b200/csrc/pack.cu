@@ -42,7 +42,9 @@ __global__ void __launch_bounds__(512) pack_kernel(const __half* __restrict__ w,
   const int lanes = G / 4;               // lanes per group
   const int gk = lane / lanes;           // this lane's group in the block
 
-  const uint2 raw = *reinterpret_cast<const uint2*>(w + n * K + (int64_t)kb * kKPerBlock + 4 * lane);
+  uint2 raw = make_uint2(0, 0);
+  if (AWQ_CHECK(in_range(n * K + (int64_t)kb * kKPerBlock + 4 * lane, 4, K * N), status))
+    raw = *reinterpret_cast<const uint2*>(w + n * K + (int64_t)kb * kKPerBlock + 4 * lane);
   const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
   const __half2 h23 = *reinterpret_cast<const __half2*>(&raw.y);
   float f[4] = {__low2float(h01), __high2float(h01), __low2float(h23), __high2float(h23)};
@@ -87,18 +89,21 @@ __global__ void __launch_bounds__(512) pack_kernel(const __half* __restrict__ w,
   // lanes 2m, 2m+1 hold inputs 8m .. 8m+7, the word word_of_k(8m) of the row
   const uint32_t word = part | __shfl_xor_sync(0xffffffffu, part, 1);
   if ((lane & 1) == 0) {
-    qweight[(block_index(nb, kb, KB, N / kRowsPerBlock) * kRowsPerBlock + r) * kWordsPerRow +
-            word_of_k(4 * lane, G)] = word;
+    const int64_t wi = (block_index(nb, kb, KB, N / kRowsPerBlock) * kRowsPerBlock + r) * kWordsPerRow +
+                       word_of_k(4 * lane, G);
+    if (AWQ_CHECK(in_range(wi, 1, K * N / 8), status)) qweight[wi] = word;
   }
   if (lane % lanes == 0) {
-    scales[((int64_t)kb * gpk + gk) * N + n] = s16;
+    if (AWQ_CHECK(in_range(((int64_t)kb * gpk + gk) * N + n, 1, K / G * N), status))
+      scales[((int64_t)kb * gpk + gk) * N + n] = s16;
     zbuf[r][gk] = zq;
   }
   __syncthreads();
   if (threadIdx.x < gpk * (kRowsPerBlock / 2)) {
     const int g = threadIdx.x / (kRowsPerBlock / 2), j = threadIdx.x % (kRowsPerBlock / 2);
-    zeros[((int64_t)kb * gpk + g) * (N / 2) + nb * (kRowsPerBlock / 2) + j] =
-        (uint8_t)(zbuf[2 * j][g] | (zbuf[2 * j + 1][g] << 4));
+    const int64_t zi = ((int64_t)kb * gpk + g) * (N / 2) + nb * (kRowsPerBlock / 2) + j;
+    if (AWQ_CHECK(in_range(zi, 1, K / G * (N / 2)), status))
+      zeros[zi] = (uint8_t)(zbuf[2 * j][g] | (zbuf[2 * j + 1][g] << 4));
   }
 }
 
@@ -118,7 +123,12 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
   const int64_t n = nb * kRowsPerBlock + r;
   const int k0 = word_k0(wi, G);
   const int64_t grow = (int64_t)kb * (kKPerBlock / G) + k0 / G;  // row of the scale / zero tables
-  const uint32_t word = qweight[block_index(nb, kb, KB, N / kRowsPerBlock) * kWordsPerBlock + t];
+  const int64_t widx = block_index(nb, kb, KB, N / kRowsPerBlock) * kWordsPerBlock + t;
+  if (!AWQ_CHECK(in_range(widx, 1, K * N / 8) && in_range(grow * N + n, 1, K / G * N) &&
+                     in_range(n * K + (int64_t)kb * kKPerBlock + k0, 8, K * N),
+                 nullptr))
+    return;
+  const uint32_t word = qweight[widx];
   const float s = __half2float(scales[grow * N + n]);
   const int z = (zeros[grow * (N / 2) + (n >> 1)] >> (4 * (n & 1))) & 0xF;
   __align__(16) __half out[8];
