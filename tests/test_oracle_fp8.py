@@ -92,6 +92,18 @@ def test_quantize_x_properties():
         # half the E4M3 spacing: 2^-4 relative for normal codes, 2^-10 sx below 2^-6
         bound = np.maximum(np.abs(xd[m]) * 2.0 ** -4, float(sx[m]) * 2.0 ** -10) * (1 + 2.0 ** -20)
         assert (np.abs(deq - xd[m]) <= bound).all()
+    # every code, element by element, is torch's E4M3 rounding of the IEEE fp32
+    # quotient x / sx (torch's float32 division and float8_e4m3fn cast, run
+    # here as a library reference); rows with sx == 0 are all-zero codes
+    live = sx > 0
+    q_t = (torch.from_numpy(x[live].astype(np.float32)) / torch.from_numpy(sx[live])[:, None]).to(torch.float8_e4m3fn)
+    assert np.array_equal(q_t.view(torch.uint8).numpy(), x8[live])
+    # on 64 x 4096 activations, where a reciprocal-multiply stand-in for the
+    # division already changes a few codes
+    xb = _x(64, 4096)
+    x8b, sxb = oracle.fp8_quantize_x(xb)
+    q_b = (torch.from_numpy(xb.astype(np.float32)) / torch.from_numpy(sxb)[:, None]).to(torch.float8_e4m3fn)
+    assert np.array_equal(q_b.view(torch.uint8).numpy(), x8b)
     # power-of-two scaling of a row changes sx by that power and no code
     x2 = (x.astype(np.float32) * 4.0).astype(np.float16)
     x8b, sxb = oracle.fp8_quantize_x(x2)

@@ -103,8 +103,9 @@ def test_every_code_is_a_nearest_grid_point(G):
     best = dist.min(axis=-1)
     mine = np.take_along_axis(dist, q[..., None].astype(np.int64), axis=-1)[..., 0]
     assert (mine == best).all()
+    # exact ties are rare in random data (the golden groups hold constructed
+    # ones); where one occurs, q - z must be even
     ties = (dist == best[..., None]).sum(axis=-1) > 1
-    assert ties.any() or True
     d = (q.astype(np.int64) - zz.astype(np.int64))[ties]
     assert (d % 2 == 0).all()
 
