@@ -144,16 +144,54 @@ def traffic_per_launch():
 # reference arm: the CPU oracle as it stands, on host cores
 # --------------------------------------------------------------------------
 
-def cpu_oracle_step(layers_packed, xs, frac):
-    """One step of the workload through the oracle, on the first `frac` of
-    every layer's output channels. Returns (algorithmic bytes covered, seconds)."""
+def host_cpu():
+    """(CPU model name, number of cores this process may run on)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    return model, cores
+
+
+def run_oracle_rows(tasks, threads):
+    """Run oracle.linear over (x, packed, N, K, n0, n1) row ranges on `threads`
+    host threads (the oracle's C code is reentrant and ctypes releases the
+    GIL while it runs); each range is split into `threads` contiguous pieces."""
+    import concurrent.futures as cf
+
     import oracle
-    t0 = time.perf_counter()
-    tot = 0.0
+    pieces = []
+    for x, hp, N, K, n0, n1 in tasks:
+        step = max(1, -(-(n1 - n0) // threads))
+        pieces += [(x, hp, N, K, a, min(n1, a + step)) for a in range(n0, n1, step)]
+    if threads == 1:
+        for x, hp, N, K, a, b in pieces:
+            oracle.linear(x, *hp, N, K, rows=(a, b))
+        return
+    with cf.ThreadPoolExecutor(threads) as ex:
+        list(ex.map(lambda t: oracle.linear(t[0], *t[1], t[2], t[3], rows=(t[4], t[5])), pieces))
+
+
+def cpu_oracle_step(layers_packed, xs, frac, threads=1):
+    """One step of the workload through the oracle, on the first `frac` of
+    every layer's output channels, on `threads` host threads. Returns
+    (algorithmic bytes covered, seconds)."""
+    tasks, tot = [], 0.0
     for (L, hp), x in zip(layers_packed, xs):
         n1 = max(16, int(L.N * frac) // 16 * 16)
-        oracle.linear(x, *hp, L.N, L.K, rows=(0, n1))
+        tasks.append((x, hp, L.N, L.K, 0, n1))
         tot += algo_bytes(M_DECODE, L.K, L.N) * n1 / L.N
+    t0 = time.perf_counter()
+    run_oracle_rows(tasks, threads)
     return tot, time.perf_counter() - t0
 
 
@@ -180,26 +218,31 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl, pool, xs = host_workload(rows=64)
-    order = [(li, r) for r in range(64) for li in range(len(pool))]
+    model, cores = host_cpu()
+    pool_rows = max(64, 16 * cores)  # output channels of each layer packed for the sample
+    wl, pool, xs = host_workload(rows=pool_rows)
     t0 = time.perf_counter()
     for li in range(len(pool)):
         Ls, hp, L = pool[li]
         oracle.linear(xs[li], *hp, Ls.N, Ls.K, rows=(0, 1))
     t_row = (time.perf_counter() - t0) / len(pool)
-    rows_per_step = int(max(1, min(len(order), args.ref_budget / (args.steps + args.warmup) / t_row)))
+    # rows of each of the four layers per step (cycling over the packed rows),
+    # split over all host cores; ~ref_budget seconds in all
+    per_layer = int(max(1, min(pool_rows, args.ref_budget * cores / (args.steps + args.warmup) / t_row / len(pool))))
     cursor = 0
 
     def one_step():
         nonlocal cursor
-        b = 0.0
-        t = time.perf_counter()
-        for _ in range(rows_per_step):
-            li, r = order[cursor % len(order)]
-            cursor += 1
+        tasks, b = [], 0.0
+        r0 = cursor % pool_rows
+        r1 = min(pool_rows, r0 + per_layer)
+        cursor = r1 % pool_rows
+        for li in range(len(pool)):
             Ls, hp, L = pool[li]
-            oracle.linear(xs[li], *hp, Ls.N, Ls.K, rows=(r, r + 1))
-            b += algo_bytes(M_DECODE, L.K, L.N) / L.N
+            tasks.append((xs[li], hp, Ls.N, Ls.K, r0, r1))
+            b += algo_bytes(M_DECODE, L.K, L.N) * (r1 - r0) / L.N
+        t = time.perf_counter()
+        run_oracle_rows(tasks, cores)
         return b, time.perf_counter() - t
 
     for _ in range(args.warmup):
@@ -210,19 +253,159 @@ def run_reference(args):
         tot_b += b
         tot_t += t
     gbs = tot_b / tot_t / 1e9
-    sample = (f"{rows_per_step} output channel(s) per step, round-robin over the first 64 rows of the four "
-              f"layers (fp64 C oracle: unpack, dequant, dot products; single thread)")
+    sample = (f"up to {per_layer} output channel(s) of each of the four layers per step, cycling over their "
+              f"first {pool_rows} rows, split over {cores} host threads (fp64 C oracle: unpack, dequant, dot products; "
+              f"CPU: {model})")
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": M_DECODE, "group": 128,
                    "layers": [[L.name, L.K, L.N] for L in wl.layers]},
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "cpu_model": model,
+                         "sample": sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# --------------------------------------------------------------------------
+# every workload configuration (GPU, rank 0 at N = 1)
+# --------------------------------------------------------------------------
+
+L2_BYTES = 126e6
+
+
+def rotations_for(weight_bytes: float, cap: int) -> int:
+    """Rotating weight copies whose total is at least 3x the L2 (every step reads HBM)."""
+    return int(max(2, min(cap, -(-3 * L2_BYTES // weight_bytes))))
+
+
+def timed_region(run, stream, min_seconds=0.25):
+    """Replays `run` (one call = one timed unit) until about `min_seconds` of
+    device time, after 3 untimed calls; CUDA events on `stream`, nvidia-smi
+    clocks sampled during the region. Returns (ms per call, calls, clocks)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(3):
+            run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    calls = int(max(10, min(20000, min_seconds * 1e3 / max(e0.elapsed_time(e1) / 3, 1e-4))))
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(calls):
+                run()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / calls, calls, clk.summary()
+
+
+def decode_sweep(awq, dev, stream, hbm):
+    """Every decode configuration: each workload's layer set as one step (one
+    awq_linear per layer), R consecutive steps over R rotating packed-weight
+    copies captured in one CUDA graph."""
+    import torch
+    out = []
+    for wl_name in ("single_4096", "llama2_7b_decode", "llama3_8b_decode", "llama2_70b_decode"):
+        wl = awq_synth.WORKLOADS[wl_name]
+        base = []
+        for L in wl.layers:
+            W = torch.from_numpy(awq_synth.layer_weight(0, wl, L).view(np.uint16)).view(torch.float16).to(dev)
+            base.append(awq.awq_pack(W, awq.new_workspace(0, L.K, L.N, dev)))
+            del W
+        wbytes = sum(algo_bytes(0, L.K, L.N) for L in wl.layers)
+        R = rotations_for(wbytes, 32)
+        packed = [base] + [[tuple(t.clone() for t in p) for p in base] for _ in range(R - 1)]
+        for M in wl.batches:
+            xs = [torch.from_numpy(awq_synth.layer_input(0, wl, L, M).view(np.uint16)).view(torch.float16).to(dev)
+                  for L in wl.layers]
+            ys = [torch.empty((M, L.N), dtype=torch.float16, device=dev) for L in wl.layers]
+            ws = torch.zeros(max(awq.awq_workspace_bytes(M, L.K, L.N) for L in wl.layers), dtype=torch.uint8,
+                             device=dev)
+
+            def steps():
+                for r in range(R):
+                    for L, x, y, p in zip(wl.layers, xs, ys, packed[r]):
+                        awq.awq_linear(x, *p, L.N, ws, y=y)
+
+            with torch.cuda.stream(stream):
+                steps()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                steps()
+            ms, calls, clocks = timed_region(g.replay, stream)
+            st = awq.awq_get_status(ws)
+            if st != awq.AWQ_OK:
+                raise RuntimeError(awq.awq_status_string(st))
+            step_bytes = sum(algo_bytes(M, L.K, L.N) for L in wl.layers)
+            us = ms * 1e3 / R
+            gbs = step_bytes / (us * 1e-6) / 1e9
+            out.append({"workload": wl_name, "M": M, "kind": "decode", "layers": [[L.name, L.K, L.N] for L in wl.layers],
+                        "us_per_step": us, "value": gbs, "unit": "GB/s", "frac": gbs / hbm,
+                        "launches_per_step": sum(awq.awq_linear_launches(M, L.K, L.N) for L in wl.layers),
+                        "rotations": R, "steps_timed": calls * R, "clocks": clocks})
+            del g, xs, ys, ws
+        del packed, base
+        torch.cuda.empty_cache()
+    return out
+
+
+def prefill_sweep(awq, dev, stream, tc_burst):
+    """Every prefill configuration, W4A16 (awq_linear: the tcgen05 GEMM) and
+    W4A8-FP8 (per-token E4M3 quantization of x + the kind::f8f6f4 GEMM), with
+    rotating packed-weight copies; eager launches (each call runs 0.05-12 ms)."""
+    import torch
+    out = []
+    wl = awq_synth.WORKLOADS["prefill"]
+    for L in wl.layers:
+        W = torch.from_numpy(awq_synth.layer_weight(0, wl, L).view(np.uint16)).view(torch.float16).to(dev)
+        base = awq.awq_pack(W, awq.new_workspace(0, L.K, L.N, dev))
+        del W
+        R = rotations_for(algo_bytes(0, L.K, L.N), 16)
+        packed = [base] + [tuple(t.clone() for t in base) for _ in range(R - 1)]
+        e8 = awq.awq_fp8_row_exponents(base[1], L.K, L.N)
+        for M in wl.batches:
+            x = torch.from_numpy(awq_synth.layer_input(0, wl, L, M).view(np.uint16)).view(torch.float16).to(dev)
+            y = torch.empty((M, L.N), dtype=torch.float16, device=dev)
+            ws = awq.new_workspace(M, L.K, L.N, dev)
+            x8 = torch.empty((M, L.K), dtype=torch.uint8, device=dev)
+            sx = torch.empty(M, dtype=torch.float32, device=dev)
+            flops = 2.0 * M * L.N * L.K
+            cur = [0]
+
+            def w4a16():
+                awq.awq_linear(x, *packed[cur[0]], L.N, ws, y=y)
+                cur[0] = (cur[0] + 1) % R
+
+            def w4a8():
+                awq.lib.awq_fp8_quantize_x(x.data_ptr(), M, L.K, x8.data_ptr(), sx.data_ptr(), stream.cuda_stream)
+                awq.awq_w4a8_gemm(x8, sx, *packed[cur[0]], e8, L.N, ws, y=y)
+                cur[0] = (cur[0] + 1) % R
+
+            for name, fn, peak in (("w4a16", w4a16, tc_burst), ("w4a8_fp8", w4a8, 2 * tc_burst)):
+                ms, calls, clocks = timed_region(fn, stream, min_seconds=0.2)
+                st = awq.awq_get_status(ws)
+                if st != awq.AWQ_OK:
+                    raise RuntimeError(awq.awq_status_string(st))
+                tf = flops / (ms * 1e-3) / 1e12
+                out.append({"workload": f"prefill/{L.name}", "K": L.K, "N": L.N, "M": M, "kind": name,
+                            "ms": ms, "value": tf, "unit": "TFLOP/s", "frac": tf / peak,
+                            "launches": awq.awq_linear_launches(M, L.K, L.N) if name == "w4a16" else None,
+                            "rotations": R, "calls_timed": calls, "clocks": clocks})
+            del x, y, ws, x8, sx
+        del packed, base, e8
+        torch.cuda.empty_cache()
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -291,33 +474,34 @@ def run_ours(args):
         for L, x, y, (qw, sc, ze) in zip(layers, xs, ys, packed[r]):
             awq.awq_linear(x, qw, sc, ze, L.N, ws, y=y)
 
-    # CUDA graphs: one graph of ROTATIONS consecutive steps (one per weight
-    # copy, 4 layers each), plus one single-step graph per copy for the steps
-    # left over when K is not a multiple of ROTATIONS
+    # CUDA graphs: graphs[j] holds j consecutive steps (weight copies 0 ..
+    # j - 1, 4 layers each); k steps replay graphs[ROTATIONS] k // ROTATIONS
+    # times, then graphs[k % ROTATIONS] once
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
         for r in range(ROTATIONS):   # warm the launch paths before capture
             step(r)
     torch.cuda.synchronize()
-    multi = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(multi, stream=stream):
-        for r in range(ROTATIONS):
-            step(r)
-    graphs = []
-    for r in range(ROTATIONS):
+    graphs = {}
+    for j in {ROTATIONS, args.steps % ROTATIONS, args.warmup % ROTATIONS} - {0}:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            step(r)
-        graphs.append(g)
+            for r in range(j):
+                step(r)
+        graphs[j] = g
     torch.cuda.synchronize()
 
     def run_steps(k):  # exactly k steps
         for _ in range(k // ROTATIONS):
-            multi.replay()
-        for r in range(k % ROTATIONS):
-            graphs[r].replay()
+            graphs[ROTATIONS].replay()
+        if k % ROTATIONS:
+            graphs[k % ROTATIONS].replay()
 
+    # every graph the warm-up and the timed region use is replayed once first,
+    # so neither region holds a graph's first launch
     with torch.cuda.stream(stream):
+        for g in graphs.values():
+            g.replay()
         run_steps(args.warmup)
     barrier()
     st = awq.awq_get_status(ws)
@@ -371,77 +555,29 @@ def run_ours(args):
            "how": "public Python API launched each step: one H2D copy of all x from pinned memory, four "
                   "awq_linear calls, one D2H copy of all y to pinned memory"}
 
-    # ---- secondary: prefill GEMM on the tensor cores ----
+    # ---- every workload configuration (rank 0 at N = 1) ----
+    sweep_decode = sweep_prefill = None
     prefill = None
-    if not args.no_prefill:
-        pwl = awq_synth.WORKLOADS[PREFILL[0]]
-        PL = pwl.layer(PREFILL[1])
-        Mp = PREFILL[2]
-        W = torch.from_numpy(awq_synth.layer_weight(0, pwl, PL).view(np.uint16)).view(torch.float16).to(dev)
-        pws = awq.new_workspace(Mp, PL.K, PL.N, dev)
-        pq = awq.awq_pack(W, pws)
-        del W
-        xp = torch.from_numpy(awq_synth.layer_input(0, pwl, PL, Mp).view(np.uint16)).view(torch.float16).to(dev)
-        yp = torch.empty((Mp, PL.N), dtype=torch.float16, device=dev)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                awq.awq_linear(xp, *pq, PL.N, pws, y=yp)
-        torch.cuda.synchronize()
-        reps = 20
-        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            p0.record(stream)
-            for _ in range(reps):
-                awq.awq_linear(xp, *pq, PL.N, pws, y=yp)
-            p1.record(stream)
-        torch.cuda.synchronize()
-        st = awq.awq_get_status(pws)
-        if st != awq.AWQ_OK:
-            raise RuntimeError(awq.awq_status_string(st))
-        pms = max_over_ranks(p0.elapsed_time(p1)) / reps
-        tflops = 2.0 * Mp * PL.N * PL.K / (pms * 1e-3) / 1e12
-        prefill = {"workload": f"{PREFILL[1]} K={PL.K} N={PL.N} M={Mp}", "ms": pms, "tflops_per_gpu": tflops,
-                   "peak_tflops": tc_burst, "frac": tflops / tc_burst, "peak_kind": f"{peak_kind} bf16 burst"}
-        # W4A8-FP8 variant on the same layer: per call, per-token E4M3
-        # quantization of x plus the kind::f8f6f4 GEMM (the row exponents are
-        # per weight, computed once like the packing)
-        e8 = awq.awq_fp8_row_exponents(pq[1], PL.K, PL.N)
-        x8 = torch.empty((Mp, PL.K), dtype=torch.uint8, device=dev)
-        sx = torch.empty(Mp, dtype=torch.float32, device=dev)
-
-        def w4a8_call():
-            awq.lib.awq_fp8_quantize_x(xp.data_ptr(), Mp, PL.K, x8.data_ptr(), sx.data_ptr(), stream.cuda_stream)
-            awq.awq_w4a8_gemm(x8, sx, *pq, e8, PL.N, pws, y=yp)
-
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                w4a8_call()
-        torch.cuda.synchronize()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            f0.record(stream)
-            for _ in range(reps):
-                w4a8_call()
-            f1.record(stream)
-        torch.cuda.synchronize()
-        st = awq.awq_get_status(pws)
-        if st != awq.AWQ_OK:
-            raise RuntimeError(awq.awq_status_string(st))
-        fms = max_over_ranks(f0.elapsed_time(f1)) / reps
-        ftf = 2.0 * Mp * PL.N * PL.K / (fms * 1e-3) / 1e12
-        prefill["w4a8_fp8"] = {"ms": fms, "tflops_per_gpu": ftf, "peak_tflops": 2 * tc_burst,
-                               "frac": ftf / (2 * tc_burst),
-                               "peak_kind": f"{peak_kind} bf16 burst x 2 (nominal dense fp8 : bf16 = 4.5 : 2.25)",
-                               "includes": "per-token E4M3 quantization of x + tcgen05 kind::f8f6f4 GEMM"}
-        del x8, sx, e8
+    if world == 1 and not args.no_sweep:
+        sweep_decode = decode_sweep(awq, dev, stream, hbm)
+        if not args.no_prefill:
+            sweep_prefill = prefill_sweep(awq, dev, stream, tc_burst)
+            pe = {(e["workload"], e["M"], e["kind"]): e for e in sweep_prefill}
+            a16, a8 = pe[(f"prefill/{PREFILL[1]}", PREFILL[2], "w4a16")], pe[(f"prefill/{PREFILL[1]}", PREFILL[2], "w4a8_fp8")]
+            prefill = {"workload": f"{PREFILL[1]} K={a16['K']} N={a16['N']} M={PREFILL[2]}", "ms": a16["ms"],
+                       "tflops_per_gpu": a16["value"], "peak_tflops": tc_burst, "frac": a16["frac"],
+                       "peak_kind": f"{peak_kind} bf16 burst", "clocks": a16["clocks"],
+                       "w4a8_fp8": {"ms": a8["ms"], "tflops_per_gpu": a8["value"], "peak_tflops": 2 * tc_burst,
+                                    "frac": a8["frac"],
+                                    "peak_kind": f"{peak_kind} bf16 burst x 2 (nominal dense fp8 : bf16 = 4.5 : 2.25)",
+                                    "includes": "per-token E4M3 quantization of x + tcgen05 kind::f8f6f4 GEMM"}}
 
     # ---- comparator: the same layers as dense fp16 weights through cuBLAS ----
-    # (torch.nn.functional.linear; a library call, timed the same way: CUDA
-    # graphs over rotating weight copies larger than L2). It gives the INT4 vs
-    # FP16 speedup the TinyChat README reports per token.
+    # (torch.matmul; a library call, timed the same way: CUDA graphs over
+    # rotating weight copies larger than L2). It gives the INT4 vs FP16
+    # speedup the TinyChat README reports per token.
     fp16 = None
     if not args.no_fp16:
-        import torch.nn.functional as F
         rot16 = 2
         w16 = [[torch.from_numpy(awq_synth.layer_weight(0, wl, L).view(np.uint16)).view(torch.float16).to(dev)
                 for L in layers] for _ in range(rot16)]
@@ -462,6 +598,8 @@ def run_ours(args):
             g16.append(g)
         steps16 = max(3, min(args.steps, 2000))
         with torch.cuda.stream(stream):
+            for g in g16:
+                g.replay()
             for i in range(args.warmup):
                 g16[i % rot16].replay()
         barrier()
@@ -475,33 +613,41 @@ def run_ours(args):
         ms16 = max_over_ranks(f0.elapsed_time(f1)) / steps16
         fp16 = {"library": "cuBLAS through torch.matmul, dense fp16 weights", "decode_ms_per_step": ms16,
                 "decode_speedup_int4_vs_fp16": ms16 / (ms / args.steps)}
-        del g16
-        del w16
+        del g16, w16
         if prefill is not None:
+            pwl = awq_synth.WORKLOADS[PREFILL[0]]
+            PL = pwl.layer(PREFILL[1])
+            Mp = PREFILL[2]
             W = torch.from_numpy(awq_synth.layer_weight(0, pwl, PL).view(np.uint16)).view(torch.float16).to(dev)
-            for _ in range(3):
-                F.linear(xp, W, out=yp)
-            torch.cuda.synchronize()
-            q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            q0.record()
-            for _ in range(20):
-                F.linear(xp, W, out=yp)
-            q1.record()
-            torch.cuda.synchronize()
-            pms16 = max_over_ranks(q0.elapsed_time(q1)) / 20
+            Ws = [W] + [W.clone() for _ in range(rotations_for(2.0 * PL.K * PL.N, 8) - 1)]
+            xp = torch.from_numpy(awq_synth.layer_input(0, pwl, PL, Mp).view(np.uint16)).view(torch.float16).to(dev)
+            yp = torch.empty((Mp, PL.N), dtype=torch.float16, device=dev)
+            cur = [0]
+
+            def mm16():
+                torch.matmul(xp, Ws[cur[0]].t(), out=yp)
+                cur[0] = (cur[0] + 1) % len(Ws)
+
+            pms16, _, _ = timed_region(mm16, stream, min_seconds=0.2)
             fp16.update({"prefill_ms": pms16, "prefill_tflops": 2.0 * Mp * PL.N * PL.K / (pms16 * 1e-3) / 1e12,
-                         "prefill_speedup_int4_vs_fp16": pms16 / prefill["ms"]})
-            del W
+                         "prefill_speedup_int4_vs_fp16": pms16 / prefill["ms"],
+                         "prefill_speedup_w4a8_vs_fp16": pms16 / prefill["w4a8_fp8"]["ms"]})
+            del W, Ws, xp, yp
         torch.cuda.empty_cache()
 
     # ---- CPU oracle baseline on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         _, hl, hx = host_workload()
-        b, t = cpu_oracle_step([(L, hp) for L, hp, _ in hl], hx, args.cpu_frac)
-        cpu = {"value": b / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"one step on the first {args.cpu_frac:.3f} of each layer's output channels "
-                         f"({t:.1f} s, fp64 C oracle, single thread)"}
+        model, cores = host_cpu()
+        lp = [(L, hp) for L, hp, _ in hl]
+        b1, t1 = cpu_oracle_step(lp, hx, args.cpu_frac / 8, threads=1)
+        b, t = cpu_oracle_step(lp, hx, args.cpu_frac, threads=cores)
+        cpu = {"value": b / t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle", "cpu_model": model,
+               "single_thread_value": b1 / t1 / 1e9,
+               "sample": f"one step on the first {args.cpu_frac:.3f} of each layer's output channels, rows split "
+                         f"over {cores} threads ({t:.1f} s); single thread: the first {args.cpu_frac / 8:.3f} of "
+                         f"the rows ({t1:.1f} s); fp64 C oracle"}
 
     traffic = traffic_per_launch()
     launches = sum(awq.awq_linear_launches(M_DECODE, L.K, L.N) for L in layers) * args.steps
@@ -513,8 +659,9 @@ def run_ours(args):
                    "layers": [[L.name, L.K, L.N] for L in layers],
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"{ROTATIONS} rotating packed-weight copies ({ROTATIONS * step_bytes / 1e6:.0f} MB > 126 MB L2)",
-                   "timing": f"CUDA graphs of {ROTATIONS} consecutive steps (one per weight copy), single-step "
-                             f"graphs for a remainder; CUDA events on the replay stream"},
+                   "timing": f"CUDA graphs of {ROTATIONS} consecutive steps (one per weight copy) and one graph "
+                             f"of the remaining steps, each replayed once before warm-up; CUDA events on the "
+                             f"replay stream"},
         "roofline": {"bound": "hbm", "achieved": per_gpu_gbs, "peak": hbm, "unit": "GB/s",
                      "frac": per_gpu_gbs / hbm, "traffic": traffic,
                      "kernel": "gemv_kernel (awq_w4a16_gemv via awq_linear)",
@@ -525,10 +672,10 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "prefill_gemm": prefill,
         "fp16_comparator": fp16,
+        "configs": (sweep_decode or []) + (sweep_prefill or []) if sweep_decode is not None else None,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del multi
     graphs.clear()
     if world > 1:
         dist.destroy_process_group()
@@ -538,6 +685,8 @@ def run_ours(args):
 SINGLE = {
     # one kernel on a layer larger than the 126 MB L2, for profiler captures
     "gemv": ("llama2_70b_decode", "gate_up", 1),     # 235 MB packed weight, M = 1
+    "gemv_7b_qkv": ("llama2_7b_decode", "qkv", 1),    # 25 MB: the decode set's second-largest layer
+    "gemv_7b_o": ("llama2_7b_decode", "o_proj", 1),   # 8 MB: the smallest, latency-bound
     "gemm": ("prefill", "llama3_gate_up", 2048),     # 58 MB weight + 16 MB x + 117 MB y
     "gemm_m512": ("prefill", "llama3_gate_up", 512),  # stream-K schedule: the GEMM and its fixup kernel
     "gemm_fp8": ("prefill", "llama3_gate_up", 2048),  # the same layer through the W4A8-FP8 GEMM
@@ -560,7 +709,7 @@ def run_single(args):
     del W
     x = torch.from_numpy(awq_synth.layer_input(0, wl, L, M).view(np.uint16)).view(torch.float16).to(dev)
     y = torch.empty((M, L.N), dtype=torch.float16, device=dev)
-    fn = awq.awq_w4a16_gemv if args.single == "gemv" else awq.awq_w4a16_gemm
+    fn = awq.awq_w4a16_gemv if args.single.startswith("gemv") else awq.awq_w4a16_gemm
     if args.single == "gemm_fp8":
         e8 = awq.awq_fp8_row_exponents(packed[1], L.K, L.N)
         x8, sx = awq.awq_fp8_quantize_x(x)
@@ -577,7 +726,7 @@ def run_single(args):
     if st != awq.AWQ_OK:
         raise RuntimeError(awq.awq_status_string(st))
     times = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.reps)]
-    work = (algo_bytes(M, L.K, L.N) / 1e9, "GB") if args.single == "gemv" else (2.0 * M * L.N * L.K / 1e12, "TFLOP")
+    work = (algo_bytes(M, L.K, L.N) / 1e9, "GB") if args.single.startswith("gemv") else (2.0 * M * L.N * L.K / 1e12, "TFLOP")
     print(json.dumps({"single": args.single, "workload": f"{wl_name}/{layer_name} K={L.K} N={L.N} M={M}",
                       "ms": times, "rate_per_s": [work[0] / (t * 1e-3) for t in times], "unit": work[1] + "/s"}))
     return 0
@@ -661,6 +810,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the per-configuration sweep (decode and prefill)")
     ap.add_argument("--no-fp16", action="store_true", help="skip the cuBLAS fp16 comparator")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-frac", type=float, default=1.0, help="share of rows in the CPU-baseline sample")
