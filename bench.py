@@ -687,6 +687,8 @@ SINGLE = {
     "gemv": ("llama2_70b_decode", "gate_up", 1),     # 235 MB packed weight, M = 1
     "gemv_7b_qkv": ("llama2_7b_decode", "qkv", 1),    # 25 MB: the decode set's second-largest layer
     "gemv_7b_o": ("llama2_7b_decode", "o_proj", 1),   # 8 MB: the smallest, latency-bound
+    "gemv_m8": ("llama3_8b_decode", "gate_up", 8),    # 61 MB, the lo/hi fp16 path at M = 8
+    "gemv_m16": ("llama3_8b_decode", "gate_up", 16),  # two token tiles
     "gemm": ("prefill", "llama3_gate_up", 2048),     # 58 MB weight + 16 MB x + 117 MB y
     "gemm_m512": ("prefill", "llama3_gate_up", 512),  # stream-K schedule: the GEMM and its fixup kernel
     "gemm_fp8": ("prefill", "llama3_gate_up", 2048),  # the same layer through the W4A8-FP8 GEMM
