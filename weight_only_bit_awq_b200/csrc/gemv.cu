@@ -67,9 +67,12 @@ constexpr int kSmemPerCta1 = 226 * 1024;
 // Byte offsets inside one ring stage for a unit of up to KU k-blocks, M
 // tokens and groups of GS inputs (the same numbers on the host and in every
 // thread). Scales, zeros and x sums hold one row per group of the unit; on
-// the integer path the x-sum slot of a k-block holds its B fragments.
+// the integer path the x-sum slot of a k-block holds its B fragments. Token
+// m's KU k-blocks of x start at x + m * xrow: the 16 pad bytes per token put
+// the eight tokens a warp's B-fragment load reads at one k on eight different
+// 16-byte bank groups (without them all eight share one: an 8-way conflict).
 struct Stage {
-  int q, s, z, xs, x, bytes;
+  int q, s, z, xs, x, xrow, bytes;
   __host__ __device__ Stage(int KU, int M, int GS, bool integer = false) {
     const int rows = KU * (kKPerBlock / GS);
     q = 0;
@@ -77,7 +80,8 @@ struct Stage {
     z = s + rows * kKbScaleBytes;
     xs = z + rows * kKbZeroBytes;
     x = xs + rows * (integer ? int_xs_bytes(M) : kKbXsBytes);
-    bytes = x + M * KU * kXRowBytes;  // every term is a multiple of 16
+    xrow = KU * kXRowBytes + 16;
+    bytes = x + M * xrow;  // every term is a multiple of 16
   }
 };
 
@@ -214,9 +218,9 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       if (lane < M) {
         // a copy that fails its check is replaced by an arrival with its byte count
         if (AWQ_CHECK(in_range((int64_t)lane * K + kb0 * kKPerBlock, (int64_t)ku * kKPerBlock, (int64_t)M * K) &&
-                          in_range(s * L.bytes + L.x + KU * kXRowBytes * lane, ku * kXRowBytes, dynamic_smem_bytes()),
+                          in_range(s * L.bytes + L.x + L.xrow * lane, ku * kXRowBytes, dynamic_smem_bytes()),
                       status))
-          ptx::bulk_g2s(sbase + s * L.bytes + L.x + KU * kXRowBytes * lane, x + (int64_t)lane * K + kb0 * kKPerBlock,
+          ptx::bulk_g2s(sbase + s * L.bytes + L.x + L.xrow * lane, x + (int64_t)lane * K + kb0 * kKPerBlock,
                         (uint32_t)(ku * kXRowBytes), xb);
 #ifdef AWQ_DEBUG
         else
@@ -271,8 +275,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
           if (m < M) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint4 v = *reinterpret_cast<const uint4*>(st + L.x + m * KU * kXRowBytes + j * kXRowBytes +
-                                                              64 * t4 + 16 * q);
+              const uint4 v = *reinterpret_cast<const uint4*>(st + L.x + m * L.xrow + j * kXRowBytes + 64 * t4 +
+                                                              16 * q);
               const float2 p0 = __half22float2(u32_as_h2(v.x)), p1 = __half22float2(u32_as_h2(v.y));
               const float2 p2 = __half22float2(u32_as_h2(v.z)), p3 = __half22float2(u32_as_h2(v.w));
               lo[j] += (p0.x + p0.y) + (p2.x + p2.y);
@@ -323,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
           uint32_t pa[KU], pb[KU], amax[KU];
 #pragma unroll
           for (int j = 0; j < KU; ++j) {
-            const uint4 xv = *reinterpret_cast<const uint4*>(st + L.x + (m * KU + j) * kXRowBytes + 16 * ch);
+            const uint4 xv = *reinterpret_cast<const uint4*>(st + L.x + m * L.xrow + j * kXRowBytes + 16 * ch);
             pa[j] = hh ? xv.y : xv.x;  // inputs (0|2, 1|3)
             pb[j] = hh ? xv.w : xv.z;  // inputs (4|6, 5|7)
             // largest fp16 magnitude of the k-block (bit patterns order like the values)
@@ -525,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       const int m = 8 * nt + g;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        xf[nt][q] = m < M ? *reinterpret_cast<const uint4*>(st + L.x + (m * KU + j) * kXRowBytes + Grp<GS>::x_off(t, q))
+        xf[nt][q] = m < M ? *reinterpret_cast<const uint4*>(st + L.x + m * L.xrow + j * kXRowBytes + Grp<GS>::x_off(t, q))
                           : make_uint4(0, 0, 0, 0);
     }
     if constexpr (kLoHi) {
@@ -615,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       const int64_t kb0 = (int64_t)jj * KU;
       const int ku = rg.KB - kb0 < KU ? (int)(rg.KB - kb0) : KU;
       if (!AWQ_CHECK(in_range(s * L.bytes + L.q, (ku * R) * 1024, dynamic_smem_bytes()) &&
-                         in_range(s * L.bytes + L.x, M * KU * kXRowBytes, dynamic_smem_bytes()),
+                         in_range(s * L.bytes + L.x, M * L.xrow, dynamic_smem_bytes()),
                      status)) {
         // (debug build) a stage that fails its check is skipped
       } else if (ku == KU) {
