@@ -281,6 +281,12 @@ awq_status awq_get_status_no_alloc(void* stream);
  * Source: none on the pages. */
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group);
 
+/* Which kernel awq_linear runs for these sizes on the current device: 1 = the
+ * decode GEMV (awq_w4a16_gemv), 2 = the tensor-core GEMM (awq_w4a16_gemm);
+ * 0 for M == 0 or invalid sizes. Host only.
+ * Source: none on the pages (dispatch query). */
+int awq_linear_path(int64_t M, int64_t K, int64_t N, int group);
+
 /* Self-test of the kernels' failure detection (the pages have no counterpart):
  * launches one thread that waits, through the same bounded-wait routine the
  * GEMM and GEMV pipelines use, on a barrier phase that nothing completes,

@@ -212,7 +212,11 @@ def test_linear_dispatch_follows_the_measured_split():
     # narrower ones. The GEMV's split-row plans launch its fixup kernel too;
     # the GEMM at M <= 32 is data-parallel (one kernel).
     assert awq.awq_linear_gemv_limit() == 16
+    assert awq.awq_linear_path(16, 4096, 28672) == 1   # GEMV
+    assert awq.awq_linear_path(24, 4096, 28672) == 2   # GEMM: 224 tiles >= 148 SMs
+    assert awq.awq_linear_path(24, 4096, 4096) == 1    # GEMV: 32 tiles
+    assert awq.awq_linear_path(32, 8192, 57344) == 2   # GEMM
+    assert awq.awq_linear_path(0, 4096, 4096) == 0
+    assert awq.awq_linear_path(1, 4000, 4096) == 0
     assert awq.awq_linear_launches(16, 4096, 28672) == 2   # GEMV + fixup
-    assert awq.awq_linear_launches(24, 4096, 28672) == 1   # GEMM: 224 tiles >= 148 SMs
-    assert awq.awq_linear_launches(24, 4096, 4096) == 2    # GEMV + fixup: 32 tiles
-    assert awq.awq_linear_launches(32, 8192, 57344) == 1   # GEMM
+    assert awq.awq_linear_launches(24, 4096, 28672) == 1   # GEMM, data-parallel

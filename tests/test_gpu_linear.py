@@ -104,8 +104,25 @@ def test_split_k_is_deterministic_and_the_workspace_reusable():
     ws = awq.new_workspace(3, K, N, xd.device)
     ys = [host(awq.awq_w4a16_gemv(xd, *dev, N, ws), np.uint16) for _ in range(3)]
     assert (ys[0] == ys[1]).all() and (ys[1] == ys[2]).all()
-    # counters were left at zero: the tail of the workspace holds no stale state
     assert awq.awq_get_status(ws) == awq.AWQ_OK
+
+
+def test_one_workspace_serves_gemv_and_stream_k_gemm_calls_of_any_size():
+    # Partial sums and stream-K parts are written before they are read, so a
+    # workspace sized for the largest call serves calls of every size and
+    # either kernel, in any order.
+    cases = [(1, 4096, 4096), (40, 1024, 38400), (3, 11008, 4096), (40, 24576, 1024), (8, 1024, 25600),
+             (1, 4096, 4096)]
+    nbytes = max(awq.awq_workspace_bytes(M, K, N) for M, K, N in cases)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    for M, K, N in cases:
+        W, dev, hp = _packed(N, K, f"share{K}x{N}")
+        x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"share{K}x{N}/x{M}"), M, K, 1.0)
+        xd = to_dev(x.view(np.uint16), torch.float16)
+        fn = awq.awq_w4a16_gemv if M <= 16 else awq.awq_w4a16_gemm
+        y = host(fn(xd, *dev, N, ws), np.float16)
+        assert awq.awq_get_status(ws) == awq.AWQ_OK
+        _check_against_oracle(y, x, hp, N, K, f"shared workspace {fn.__name__} M={M} K={K} N={N}")
 
 
 def test_gemv_and_gemm_agree_closely():

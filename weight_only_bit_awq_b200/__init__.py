@@ -9,7 +9,7 @@ importing the binding fails loudly if the shared library cannot be loaded.
 Functions (same names as the C entry points):
   awq_packed_size, awq_workspace_bytes, awq_workspace_init, awq_pack,
   awq_dequant, awq_w4a16_gemv, awq_w4a16_gemm, awq_linear,
-  awq_linear_gemv_limit, awq_linear_launches, awq_check_bounded_wait,
+  awq_linear_gemv_limit, awq_linear_launches, awq_linear_path, awq_check_bounded_wait,
   awq_get_status, awq_status_string, awq_w4a16_gemv_no_alloc,
   awq_get_status_no_alloc, and the W4A8-FP8
   variant awq_fp8_row_exponents, awq_fp8_quantize_x, awq_dequant_fp8,
@@ -41,6 +41,7 @@ globals().update({name: code for code, name in STATUS_NAMES.items()})
 EXPORTS = ("awq_packed_size", "awq_workspace_bytes", "awq_workspace_init", "awq_pack", "awq_dequant",
            "awq_w4a16_gemv", "awq_w4a16_gemm", "awq_linear", "awq_linear_gemv_limit", "awq_get_status",
            "awq_status_string", "awq_w4a16_gemv_no_alloc", "awq_get_status_no_alloc", "awq_linear_launches",
+           "awq_linear_path",
            "awq_check_bounded_wait",
            "awq_fp8_row_exponents", "awq_fp8_quantize_x", "awq_dequant_fp8", "awq_w4a8_gemm")
 
@@ -83,6 +84,7 @@ def _load() -> ctypes.CDLL:
     lib.awq_get_status_no_alloc.argtypes = [vp]
     lib.awq_linear_gemv_limit.argtypes = []
     lib.awq_linear_launches.argtypes = [i64, i64, i64, ci]
+    lib.awq_linear_path.argtypes = [i64, i64, i64, ci]
     lib.awq_check_bounded_wait.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.awq_get_status.argtypes = [vp, vp]
     lib.awq_fp8_row_exponents.argtypes = [vp, i64, i64, ci, vp, vp]
@@ -270,6 +272,11 @@ def awq_linear_gemv_limit() -> int:
 def awq_linear_launches(M: int, K: int, N: int, group: int = GROUP) -> int:
     """Kernels awq_linear launches for these sizes on the current device."""
     return int(lib.awq_linear_launches(M, K, N, group))
+
+
+def awq_linear_path(M: int, K: int, N: int, group: int = GROUP) -> int:
+    """Kernel awq_linear runs for these sizes: 1 = the GEMV, 2 = the GEMM, 0 = none."""
+    return int(lib.awq_linear_path(M, K, N, group))
 
 
 def awq_check_bounded_wait(workspace: torch.Tensor, limit_us: int = 1000):

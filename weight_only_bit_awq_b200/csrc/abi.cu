@@ -330,6 +330,11 @@ awq_status awq_w4a8_gemm(const void* x8, const void* sx, const void* qweight, co
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
+int awq_linear_path(int64_t M, int64_t K, int64_t N, int group) {
+  if (M <= 0 || M > kMaxM || check_kn(K, N, group) != AWQ_OK) return 0;
+  return linear_uses_gemv(M, N, sm_count_or_default()) ? 1 : 2;
+}
+
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group) {
   if (M <= 0 || M > kMaxM || check_kn(K, N, group) != AWQ_OK) return 0;
   const int sms = sm_count_or_default();

@@ -21,7 +21,7 @@
 //     and one bulk copy per token of x[m][128 kb0 .. 128 (kb0 + KU)); the
 //     stage's mbarrier tracks completion (transaction bytes plus the cp.async
 //     arrivals). The ring depth follows from the shared memory left for the
-//     stage size. The codes of the first stages are requested before the
+//     stage size. The codes of the first stage are requested before the
 //     kernel waits for the previous grid in the stream (programmatic
 //     dependent launch): they do not depend on it; x does.
 //   warps 1-8 (consumers): warp w owns row block w of every unit, so it
@@ -230,10 +230,20 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
       }
       if (++xj == rg.UPG) xj = 0;
     };
+    // Only the first stage's codes go out before the previous grid has
+    // finished (they do not depend on it). Every CTA asking for its whole ring
+    // at once puts tens of MB in the memory queues, and the loads that the
+    // previous layer's fixup and this layer's x wait for then queue behind
+    // them: measured on B200, one stage ahead is 6-9% faster per decode layer
+    // set than a full ring, and two stages sit in between.
     const int pro = n_units < NS ? n_units : NS;
-    for (int i = 0; i < pro; ++i) issue_codes(i);  // independent of the previous grid
+    if (pro > 0) issue_codes(0);
     ptx::griddep_wait();
-    for (int i = 0; i < pro; ++i) issue_x(i);
+    if (pro > 0) issue_x(0);
+    for (int i = 1; i < pro; ++i) {
+      issue_codes(i);
+      issue_x(i);
+    }
     // unit i goes to stage s = i % NS as its use ph = (i / NS) & 1 and waits
     // for the consumers' release of the stage's previous use (parity ph ^ 1)
     int i = pro, s = pro % NS, ph = pro / NS;
