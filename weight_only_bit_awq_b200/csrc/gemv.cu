@@ -515,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
   using Acc = std::conditional_t<kLoHi, float[LoHi<GS>::kAcc][4], float[kC][NT][4]>;
   struct KState {
     float s[kGPK][2];     // scales of rows g, g + 8 per group of the k-block
-    float corr[kGPK][4];  // lo/hi path: s (C + z X) of slot cc (rows g / g+8, tokens 2t / 2t+1)
+    float corr[kGPK][4];  // lo/hi path: C + z X of slot cc (rows g / g+8, tokens 2t / 2t+1)
   };
   auto kb_issue = [&](const uint8_t* st, int j, int R, Acc& acc, KState& ks) {
     const uint8_t* blk = st + L.q + (j * R + cw) * 1024;
@@ -554,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
         for (int cc = 0; cc < 4; ++cc) {
           if (kM1 && (cc & 1)) continue;  // slots of token 1
           const float Cm = (cc & 1) ? cx.z : cx.x, Xm = (cc & 1) ? cx.w : cx.y;
-          ks.corr[gk][cc] = ks.s[gk][cc >> 1] * fmaf(zf[cc >> 1], Xm, Cm);
+          ks.corr[gk][cc] = fmaf(zf[cc >> 1], Xm, Cm);
         }
       }
     } else {
@@ -563,16 +563,14 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
   };
   auto kb_finish = [&](const Acc& acc, const KState& ks) {
     if constexpr (kLoHi) {
-      // y += s (acc_lo + acc_hi / 16) - s (C + z X), per group
-      constexpr int kLo = LoHi<GS>::kLo;
+      // y += s (acc - (C + z X)), per group
 #pragma unroll
       for (int gk = 0; gk < kGPK; ++gk)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           if (kM1 && (cc & 1)) continue;
-          const float lo = GS == 128 ? acc[0][cc] + acc[1][cc] : acc[gk][cc];
-          const float hi = GS == 128 ? acc[2][cc] + acc[3][cc] : acc[kLo + gk][cc];
-          yacc[0][cc] = fmaf(ks.s[gk][cc >> 1], fmaf(hi, 0.0625f, lo), yacc[0][cc]) - ks.corr[gk][cc];
+          const float a = GS == 128 ? acc[0][cc] + acc[1][cc] : acc[gk][cc];
+          yacc[0][cc] = fmaf(ks.s[gk][cc >> 1], a - ks.corr[gk][cc], yacc[0][cc]);
         }
     } else {
 #pragma unroll

@@ -142,44 +142,43 @@ __device__ __forceinline__ float pos_half_bits_to_float(uint32_t h) {
   return __uint_as_float(h << 13) * 5.192296858534828e+33f;  // 2^112; the sign bit of h is 0
 }
 
-// M <= 8 (one token tile): the codes go into the MMA unchanged, as the fp16
-// values 1024 + q (pairs taken with the 0x000F000F mask, "lo" k) and
-// 1024 + 16 q (0x00F000F0 mask, "hi" k), in separate MMAs so that the two
-// offsets can be removed afterwards with per-group sums of x:
-//   sum_k x (q - z) = acc_lo + acc_hi / 16 - (1024 X_lo + 64 X_hi) - z (X_lo + X_hi)
+// M <= 8 (one token tile): the codes go into the MMA unchanged. One lop3
+// turns the nibbles at bits 0-3 of each half of a word ("lo" k) into the fp16
+// values 1024 + q (0x000F000F mask over 0x6400 = 1024, whose ulp is 1), and
+// the nibbles at bits 4-7 ("hi" k) into 64 + q (0x00F000F0 mask over 0x5400 =
+// 64, whose ulp is 1/16, so mantissa 16 q adds q). Both kinds accumulate in
+// the same fp32 registers, and the offsets come off afterwards with per-group
+// sums of x:
+//   sum_k x (q - z) = acc - (1024 X_lo + 64 X_hi) - z (X_lo + X_hi)
 // with X_lo, X_hi the sums of x over the lo and hi k of the group. This needs
 // 5 integer ops per 8 weights and no fp16 arithmetic. LoHi<GS>::kAcc
-// accumulators: lo ones first, then hi ones; for GS = 128 two chains of each,
-// else one of each per group.
+// accumulators: for GS = 128 two chains (alternate MMA steps), else one per
+// group.
 template <int GS>
 struct LoHi {
-  static constexpr int kLo = GS == 128 ? 2 : Grp<GS>::kPerKb;
-  static constexpr int kAcc = 2 * kLo;
+  static constexpr int kAcc = GS == 128 ? 2 : Grp<GS>::kPerKb;
 };
 template <int GS>
 __device__ __forceinline__ void block_mma_lohi(float (&acc)[LoHi<GS>::kAcc][4], const uint4& wa4, const uint4& wb4,
                                                const uint4 (&xf)[4]) {
-  constexpr int kLo = LoHi<GS>::kLo, J = Grp<GS>::J;
-  const uint32_t kMaskLo = 0x000F000Fu, kMaskHi = 0x00F000F0u, kMagic = 0x64006400u;
+  constexpr int J = Grp<GS>::J;
+  const uint32_t kMaskLo = 0x000F000Fu, kMaskHi = 0x00F000F0u, kMagicLo = 0x64006400u, kMagicHi = 0x54005400u;
   const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
   const uint32_t wb[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t a = wa[j], b = wb[j], a8 = wa[j] >> 8, b8 = wb[j] >> 8;
     // slots (2t, 2t+1) <- k0 + 0, 1 (lo) / 2, 3 (hi); slots (2t+8, 2t+9) <- k0 + 4, 5 / 6, 7
-    const uint32_t l0 = lop3_and_or(a, kMaskLo, kMagic), l1 = lop3_and_or(b, kMaskLo, kMagic);
-    const uint32_t l2 = lop3_and_or(a8, kMaskLo, kMagic), l3 = lop3_and_or(b8, kMaskLo, kMagic);
-    const uint32_t h0 = lop3_and_or(a, kMaskHi, kMagic), h1 = lop3_and_or(b, kMaskHi, kMagic);
-    const uint32_t h2 = lop3_and_or(a8, kMaskHi, kMagic), h3 = lop3_and_or(b8, kMaskHi, kMagic);
+    const uint32_t l0 = lop3_and_or(a, kMaskLo, kMagicLo), l1 = lop3_and_or(b, kMaskLo, kMagicLo);
+    const uint32_t l2 = lop3_and_or(a8, kMaskLo, kMagicLo), l3 = lop3_and_or(b8, kMaskLo, kMagicLo);
+    const uint32_t h0 = lop3_and_or(a, kMaskHi, kMagicHi), h1 = lop3_and_or(b, kMaskHi, kMagicHi);
+    const uint32_t h2 = lop3_and_or(a8, kMaskHi, kMagicHi), h3 = lop3_and_or(b8, kMaskHi, kMagicHi);
     const int idx = GS == 128 ? (j & 1) : j / J;
-    const bool first = GS == 128 ? j < 2 : j % J == 0;
-    if (first) {
+    if (GS == 128 ? j < 2 : j % J == 0)
       mma_16816_first(acc[idx], l0, l1, l2, l3, xf[j].x, xf[j].z);
-      mma_16816_first(acc[kLo + idx], h0, h1, h2, h3, xf[j].y, xf[j].w);
-    } else {
+    else
       mma_16816(acc[idx], l0, l1, l2, l3, xf[j].x, xf[j].z);
-      mma_16816(acc[kLo + idx], h0, h1, h2, h3, xf[j].y, xf[j].w);
-    }
+    mma_16816(acc[idx], h0, h1, h2, h3, xf[j].y, xf[j].w);
   }
 }
 
