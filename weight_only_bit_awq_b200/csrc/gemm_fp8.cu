@@ -429,19 +429,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int g = 0; g < kGPK; ++g) gc[g] = group_consts(sb[g], z[g], pow2e);
         uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
+        // Word ww of code chunk cj = 2 hf + cl (cl = 0, 1; held by c[cl ^ rot])
+        // holds inputs k0 .. k0 + 7 with k0 = GS (ww / J) + 8 (cj J + ww % J),
+        // i.e. half k0 & 8 of 16-input chunk k0 / 16 of the row. The thread's
+        // eight words fill four whole chunks, which go out as four 16-byte
+        // stores; at a fixed store the 32 lanes (16 rows x 2 halves) hit the
+        // eight swizzled chunk positions four times each (no bank conflict).
+        // (Eight-byte stores left half of each chunk's banks idle per store:
+        // 4x the ideal wavefronts at groups of 128.)
+        constexpr int J = GS / 32;
+        uint4 out[4];
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int cj = 2 * hf + ((jj + rot) & 1);  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
-          const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
+        for (int cl = 0; cl < 2; ++cl) {
+          const uint4 cw = rot ? c[cl ^ 1] : c[cl];
+          const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
           for (int ww = 0; ww < 4; ++ww) {
-            // word 4 cj + ww holds inputs k0 .. k0 + 7 of group ww / (GS / 32)
-            constexpr int J = GS / 32;
-            const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
-            const int chunk = k0 >> 4;  // 16-byte chunk (16 inputs) of the 128-byte row
-            *reinterpret_cast<uint2*>(wt + ((chunk ^ (row & 7)) << 4) + (k0 & 8)) =
-                w8_word(words[ww], gc[g].zlo, gc[g].zhi, gc[g].s2);
+            const int g = ww / J;
+            const uint2 v = w8_word(words[ww], gc[g].zlo, gc[g].zhi, gc[g].s2);
+            // slot (chunk among the thread's four) and half of this word
+            const int slot = GS == 128 ? 2 * cl + (ww >> 1) : (GS == 64 ? 2 * (ww >> 1) + cl : ww);
+            const int hi = GS == 32 ? cl : (ww & 1);
+            if (hi) {
+              out[slot].z = v.x;
+              out[slot].w = v.y;
+            } else {
+              out[slot].x = v.x;
+              out[slot].y = v.y;
+            }
           }
+        }
+#pragma unroll
+        for (int slot = 0; slot < 4; ++slot) {
+          const int chunk = GS == 128 ? 4 * hf + slot : (GS == 64 ? 4 * (slot >> 1) + 2 * hf + (slot & 1) : 2 * slot + hf);
+          *reinterpret_cast<uint4*>(wt + ((chunk ^ (row & 7)) << 4)) = out[slot];
         }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(bar(kBarWFull + ws));
