@@ -442,3 +442,39 @@ def test_gemm_small_m_many_tiles(M, K, N, group):
     rows = sample_rows(N, 256, seed=M)
     y_ref, b = oracle_rows(x, *hp, N, K, rows, group)
     check_close(ys[0][:, rows], y_ref, b, f"gemm M={M} K={K} N={N} group={group}")
+
+
+# ---- prefill GEMM on CTA pairs (tcgen05 cta_group::2) ------------------------
+# The data-parallel schedule at 256-token tiles runs on clusters of two CTAs
+# that share one MMA stream: 256 channels x 256 tokens per tile, each CTA
+# dequantizing its 128 channels and loading its 128 tokens. Shapes (M, K, N,
+# group): an even number of channel tiles; an odd one (the last pair has one
+# CTA without channels) with a ragged last token tile; groups of 64 and 32.
+PAIR_CASES = [(512, 256, 16384, 128), (500, 256, 16512, 128), (512, 256, 16384, 64), (512, 256, 16384, 32)]
+
+
+@pytest.mark.parametrize("M,K,N,group", PAIR_CASES)
+def test_gemm_cta_pairs_match_oracle(M, K, N, group):
+    W, dev, hp = _packed(N, K, f"pair{K}x{N}", group=group)
+    x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"pair{K}x{N}/x{M}"), M, K, 1.0)
+    xd = to_dev(x.view(np.uint16), torch.float16)
+    ws = awq.new_workspace(M, K, N, xd.device, group)
+    ys = [host(awq.awq_w4a16_gemm(xd, *dev, N, ws, group), np.float16) for _ in range(2)]
+    assert awq.awq_get_status(ws) == awq.AWQ_OK
+    assert (ys[0].view(np.uint16) == ys[1].view(np.uint16)).all()  # deterministic
+    _check_against_oracle(ys[0], x, hp, N, K, f"pair gemm M={M} K={K} N={N} G={group}", group=group)
+
+
+def test_gemm_cta_pairs_one_hot_gives_every_dequantized_weight():
+    # every output channel of both CTAs of every pair, bit for bit
+    M, K, N = 512, 256, 16512
+    W, dev, hp = _packed(N, K, "pair1hot")
+    x = np.zeros((M, K), np.float16)
+    ks = [(37 * m + 11) % K for m in range(M)]
+    for m, k in enumerate(ks):
+        x[m, k] = 1.0
+    y = _run(awq.awq_w4a16_gemm, x, dev, N)
+    q, z, s = oracle.unpack(*hp, N, K)
+    wh = oracle.dequant(q, z, s)
+    for m, k in enumerate(ks):
+        assert (y[m].view(np.uint16) == wh[:, k].view(np.uint16)).all(), (m, k)

@@ -108,6 +108,7 @@ struct GemmPlan {
   int ctas;             // persistent CTAs (at most one per SM)
   int dp_tiles;         // the first dp_tiles tiles are computed whole, data-parallel
   bool stream_k;        // the other tiles' k-blocks are split over the CTAs; the fixup kernel runs
+  bool pair;            // data-parallel at 256-token tiles on CTA pairs (gemm_pair_kernel)
   size_t partial_off;   // workspace offset of the split tiles' fp32 parts (bytes)
   size_t ws_bytes;      // total workspace bytes
 };

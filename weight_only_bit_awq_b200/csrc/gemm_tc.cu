@@ -441,6 +441,321 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// CTA pairs (tcgen05 cta_group::2): tiles of 256 output channels x 256 tokens
+// ---------------------------------------------------------------------------
+// A cluster of two CTAs computes one 256-channel x 256-token tile with a
+// single stream of tcgen05.mma issued by CTA 0 of the pair (the leader). CTA
+// r dequantizes channel tile 2 np + r (its 128 rows of A) and loads tokens
+// m0 + 128 r .. m0 + 128 r + 127 of x (its half of B); each MMA reads both
+// CTAs' shared memory and accumulates each CTA's 128 rows x 256 tokens in that
+// CTA's tensor memory. At the flops per SM of the one-CTA kernel, each SM holds
+// and feeds the tensor core only half of the x tile, so the x ring is twice as
+// deep in the same shared memory.
+// Barriers: the leader's x-full barrier expects both halves' bytes, and both
+// CTAs' TMA loads complete on it; the leader's W-full and accumulator-empty
+// barriers count the dequant and epilogue threads of both CTAs, which arrive
+// across the cluster; the MMA's commits arrive on the x-empty, W-empty and
+// accumulator-full barriers of both CTAs (multicast commit). Code stages stay
+// per CTA. Used for the data-parallel schedule at 256-token tiles (no
+// stream-K), the large prefill shapes.
+struct PairLayout {
+  static constexpr int kHalfBN = 128;  // tokens of x per CTA
+  static constexpr int kXStages = 6, kWStages = 3, kQStages = 2;
+  static_assert(kQStages % 2 == 0, "each code stage belongs to one dequant group");
+  static constexpr int kBarXFull = 0, kBarXEmpty = kBarXFull + kXStages, kBarWFull = kBarXEmpty + kXStages,
+                       kBarWEmpty = kBarWFull + kWStages, kBarQFull = kBarWEmpty + kWStages,
+                       kBarQEmpty = kBarQFull + kQStages, kBarAccFull = kBarQEmpty + kQStages,
+                       kBarAccEmpty = kBarAccFull + 2, kBarDrain = kBarAccEmpty + 2, kNumBars = kBarDrain + 1;
+  static constexpr int kXBytes = kHalfBN * 64 * 2;
+  static constexpr int kXOff = 0;
+  static constexpr int kWOff = kXOff + kXStages * kXBytes;
+  static constexpr int kQOff = kWOff + kWStages * kWBytes;
+  static constexpr int kBarOff = kQOff + kQStages * kQStride;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1 KiB
+};
+static_assert(PairLayout::kAlloc <= 232448, "shared memory budget");
+
+// Pair tiles t = cl, cl + P2, ... of cluster cl (P2 clusters): tile_coords over
+// token tiles x channel-tile pairs; this CTA's channel tile is 2 np + rank.
+template <int GS>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
+                     const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y,
+                     int M, int K, int N, int GM, uint32_t* status) {
+  using L = PairLayout;
+  constexpr int BN = 256;
+  constexpr int kXStages = L::kXStages, kWStages = L::kWStages, kQStages = L::kQStages;
+  constexpr int kBarXFull = L::kBarXFull, kBarXEmpty = L::kBarXEmpty, kBarWFull = L::kBarWFull,
+                kBarWEmpty = L::kBarWEmpty, kBarQFull = L::kBarQFull, kBarQEmpty = L::kBarQEmpty,
+                kBarAccFull = L::kBarAccFull, kBarAccEmpty = L::kBarAccEmpty, kBarDrain = L::kBarDrain;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBarOff + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int KB = K / kKPerBlock;
+  const int MT = (M + BN - 1) / BN, NT = (N + kBM - 1) / kBM, NP = (NT + 1) / 2, T2 = MT * NP;
+  const int P2 = (int)gridDim.x / 2, cl = (int)blockIdx.x / 2;
+  const int ntiles = cl < T2 ? (T2 - 1 - cl) / P2 + 1 : 0;
+  auto tile = [&](int j, int& mt, int& nt) {
+    int np;
+    tile_coords(cl + j * P2, MT, NP, GM, mt, np);
+    nt = 2 * np + (int)rank;  // >= NT: no channels (the last pair when NT is odd)
+  };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kXStages; ++i) {
+      ptx::mbar_init(bar(kBarXFull + i), 1);   // the leader's expect_tx (both halves' bytes)
+      ptx::mbar_init(bar(kBarXEmpty + i), 1);  // one commit
+    }
+    for (int i = 0; i < kWStages; ++i) {
+      ptx::mbar_init(bar(kBarWFull + i), kDeqThreads);  // one dequant group in each CTA of the pair
+      ptx::mbar_init(bar(kBarWEmpty + i), 1);
+    }
+    for (int i = 0; i < kQStages; ++i) {
+      ptx::mbar_init(bar(kBarQFull + i), 33);
+      ptx::mbar_init(bar(kBarQEmpty + i), kDeqThreads / 2);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(kBarAccFull + i), 1);
+      ptx::mbar_init(bar(kBarAccEmpty + i), 2 * kEpiThreads);  // the epilogue threads of both CTAs
+    }
+    ptx::mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == kWarpX && lane == 0) ptx::prefetch_tensormap(&tmap_x);
+  if (warp == kWarpMma) {
+    ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), 2 * BN);
+    ptx::tmem_relinquish_pair();
+    ptx::tc_fence_before();
+  }
+  __syncthreads();
+  ptx::cluster_sync();  // both CTAs' barriers exist before any arrive crosses the pair
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  auto lead = [&](int i) -> uint32_t { return ptx::mapa(bar(i), 0); };  // the leader's barrier i
+
+  if (warp == kWarpX) {
+    // ---------------- x producer: this CTA's 128 tokens, 2 boxes of 64 k per k-block ----------------
+    if (lane == 0) {
+      int i = 0;
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        int mt, nt;
+        tile(j, mt, nt);
+        const int m0 = mt * BN + L::kHalfBN * (int)rank;
+        for (int h = 0; h < 2 * KB; ++h, ++i) {
+          const int s = i % kXStages;
+          if (!(ok = wait_bar(bar(kBarXEmpty + s), ((i / kXStages) & 1) ^ 1, abort_flag, status))) break;
+          if (leader) ptx::mbar_arrive_expect_tx(bar(kBarXFull + s), 2 * L::kXBytes);
+          ptx::tma_load_2d_pair(sbase + L::kXOff + s * L::kXBytes, &tmap_x, h * 64, m0, lead(kBarXFull + s));
+        }
+      }
+      if (!ok) {
+        if (leader) {  // aborting: let the copies the leader's barriers count land
+          for (int j = (i > kXStages ? i - kXStages : 0); j < i; ++j)
+            drain_bar(bar(kBarXFull + j % kXStages), (j / kXStages) & 1);
+        } else {  // the peer's copies count on the leader's barriers: give them time to land
+          const uint64_t t0 = ptx::globaltimer_ns();
+          while (ptx::globaltimer_ns() - t0 < ptx::kDrainLimitNs) {
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kWarpQ) {
+    // ---------------- packed-weight producer (this CTA's channel tile) ----------------
+    constexpr int kGPK = kKPerBlock / GS;
+    const int64_t NB = N / kRowsPerBlock;
+    int i = 0;
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      int mt, nt;
+      tile(j, mt, nt);
+      const bool has = nt < NT;
+      const int64_t gi = nt;
+      const int n0 = nt * kBM;
+      const uint32_t qbytes = has ? (uint32_t)(group_rows(gi, NB) * 1024) : 0u;
+      for (int kb = 0; kb < KB; ++kb, ++i) {
+        const int s = i % kQStages;
+        if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((i / kQStages) & 1) ^ 1, abort_flag, status);
+        if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+        const uint32_t st = sbase + L::kQOff + s * kQStride;
+        const int64_t qw0 = has ? unit_first_block(gi, kb, KB, NB) * kWordsPerBlock : 0;
+        const bool qok = qbytes > 0 && AWQ_CHECK(in_range(qw0, qbytes / 4, (int64_t)K * N / 8), status);
+        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qok ? qbytes : 0u);
+        __syncwarp();
+        if (lane == 0 && qok) ptx::bulk_g2s(st, qweight + qw0, qbytes, bar(kBarQFull + s));
+        for (int p = lane; p < kGPK * 16; p += 32) {
+          const int g = p >> 4, l = p & 15;
+          if (n0 + 8 * l < N &&
+              AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * N + n0 + 8 * l, 8, (int64_t)(K / GS) * N), status))
+            ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
+        }
+        for (int p = lane; p < kGPK * 8; p += 32) {
+          const int g = p >> 3, l = p & 7;
+          if (n0 + 16 * l < N &&
+              AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l, 8, (int64_t)(K / GS) * (N / 2)),
+                        status))
+            ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l,
+                            zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
+        }
+        ptx::cp_async_arrive_noinc(bar(kBarQFull + s));
+      }
+    }
+    if (!ok && lane == 0)
+      for (int j = (i > kQStages ? i - kQStages : 0); j < i; ++j)
+        drain_bar(bar(kBarQFull + j % kQStages), (j / kQStages) & 1);
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    // ---------------- MMA issuer (the leader only) ----------------
+    if (leader && lane == 0) {
+      const uint32_t idesc = ptx::idesc_f16_f32(2 * kBM, BN);  // M = 256 over the pair
+      bool ok = true;
+      int wi = 0, xi = 0;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int acc = j & 1;
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        if (!(ok = wait_bar(bar(kBarAccEmpty + acc), ((j >> 1) & 1) ^ 1, abort_flag, status))) break;
+        ptx::tc_fence_after();
+        for (int kb = 0; kb < KB && ok; ++kb, ++wi) {
+          const int ws = wi % kWStages;
+          if (!(ok = wait_bar(bar(kBarWFull + ws), (wi / kWStages) & 1, abort_flag, status))) break;
+          ptx::tc_fence_after();
+          for (int h = 0; h < 2; ++h, ++xi) {
+            const int s = xi % kXStages;
+            if (!(ok = wait_bar(bar(kBarXFull + s), (xi / kXStages) & 1, abort_flag, status))) break;
+            ptx::tc_fence_after();
+            const uint32_t a_base = sbase + L::kWOff + ws * kWBytes + h * kWHalfBytes;
+            const uint32_t b_base = sbase + L::kXOff + s * L::kXBytes;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              ptx::mma_f16_ss_pair(d_tmem, ptx::desc_kmajor_sw128(a_base + 32 * kk),
+                                   ptx::desc_kmajor_sw128(b_base + 32 * kk), idesc, (kb | h | kk) != 0);
+            ptx::mma_commit_pair(bar(kBarXEmpty + s));
+          }
+          if (ok) ptx::mma_commit_pair(bar(kBarWEmpty + ws));
+        }
+        if (ok) ptx::mma_commit_pair(bar(kBarAccFull + acc));
+      }
+      if (!ok) {  // aborting: wait for the MMAs already issued
+        ptx::mma_commit_pair(bar(kBarDrain));
+        drain_bar(bar(kBarDrain), 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp < kFirstEpiWarp) {
+    // ---------------- dequantize (as in gemm_kernel; W-full is the leader's) ----------------
+    const int d = threadIdx.x - kFirstDeqWarp * 32;
+    const int grp = d >> 7, row = d & (kBM - 1);
+    const int rot = (row >> 1) & 3;
+    constexpr int kGPK = kKPerBlock / GS;
+    bool ok = true;
+    int i = 0;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      for (int kb = 0; kb < KB; ++kb, ++i) {
+        if ((i & 1) != grp) continue;
+        const int qs = i % kQStages;
+        if (!(ok = wait_bar(bar(kBarQFull + qs), (i / kQStages) & 1, abort_flag, status))) break;
+        const uint8_t* qst = smem + L::kQOff + qs * kQStride;
+        const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64;
+        uint4 c[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 3));
+        uint32_t s[kGPK], z[kGPK];
+#pragma unroll
+        for (int g = 0; g < kGPK; ++g) {
+          s[g] = reinterpret_cast<const uint16_t*>(qst + kQScaleOff + 256 * g)[row];
+          z[g] = (qst[kQZeroOff + 64 * g + (row >> 1)] >> (4 * (row & 1))) & 0xF;
+        }
+        ptx::mbar_arrive(bar(kBarQEmpty + qs));
+
+        const int ws = i % kWStages;
+        if (!(ok = wait_bar(bar(kBarWEmpty + ws), ((i / kWStages) & 1) ^ 1, abort_flag, status))) break;
+        __half2 s2[kGPK], zlo[kGPK], zhi[kGPK];
+#pragma unroll
+        for (int g = 0; g < kGPK; ++g) {
+          s2[g] = u2h(s[g] * 0x00010001u);
+          zlo[g] = u2h((0x6400u + z[g]) * 0x00010001u);
+          zhi[g] = u2h((0xD400u + (z[g] << 4)) * 0x00010001u);
+        }
+        uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int cj = (jj + rot) & 3;
+          const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
+#pragma unroll
+          for (int ww = 0; ww < 4; ++ww) {
+            constexpr int J = GS / 32;
+            const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
+            const int chunk = (k0 & 63) >> 3;
+            uint8_t* dst = wt + (k0 >> 6) * kWHalfBytes;
+            *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) =
+                dequant_word(words[ww], zlo[g], zhi[g], s2[g]);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        if (leader)
+          ptx::mbar_arrive(bar(kBarWFull + ws));
+        else
+          ptx::mbar_arrive_cluster(lead(kBarWFull + ws));
+      }
+    }
+  } else {
+    // ---------------- epilogue: this CTA's 128 channels x 256 tokens ----------------
+    const int quad = warp & 3;
+    const int r = 32 * quad + lane;
+    for (int j = 0; j < ntiles; ++j) {
+      int mt, nt;
+      tile(j, mt, nt);
+      const int acc = j & 1;
+      if (!wait_bar(bar(kBarAccFull + acc), (j >> 1) & 1, abort_flag, status)) break;
+      ptx::tc_fence_after();
+      const int m0 = mt * BN, nn = nt * kBM + r;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        if (m0 + c0 >= M) break;
+        uint32_t v[16];
+        ptx::tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * BN + c0), v);
+        ptx::tmem_wait_ld();
+        if (nt < NT && nn < N) {
+#pragma unroll
+          for (int q = 0; q < 16; q += 2) {
+            const int m = m0 + c0 + q;
+            const __half2 h = __floats2half2_rn(__uint_as_float(v[q]), __uint_as_float(v[q + 1]));
+            if (m < M && AWQ_CHECK(in_range((int64_t)m * N + nn, 1, (int64_t)M * N), status))
+              y[(int64_t)m * N + nn] = __low2half(h);
+            if (m + 1 < M && AWQ_CHECK(in_range((int64_t)(m + 1) * N + nn, 1, (int64_t)M * N), status))
+              y[(int64_t)(m + 1) * N + nn] = __high2half(h);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      if (leader)
+        ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+      else
+        ptx::mbar_arrive_cluster(lead(kBarAccEmpty + acc));
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // the pair's MMAs, copies and tensor-memory reads are done in both CTAs
+  if (warp == kWarpMma) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem_base, 2 * BN);
+  }
+}
+
 // Stream-K tiles split between CTAs: CTA (s, b) adds the parts of stream-K
 // tile s, token columns 32 b .. 32 b + 31, thread = channel row of the tile.
 // The contributors are the CTAs whose k-block ranges meet the tile's, in CTA
@@ -554,10 +869,85 @@ cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* sc
                             p.gm, p.dp_tiles, p.ctas, part_floats, status);
 }
 
+// Pair clusters that can be resident at once on device `dev` (0 if none): the
+// grid of gemm_pair_kernel, cached per device.
+template <int GS>
+int pair_clusters(int dev) {
+  static std::atomic<int> cache[64];
+  int n = cache[dev].load(std::memory_order_acquire);
+  if (n != 0) return n > 0 ? n : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = PairLayout::kAlloc;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel<GS>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    clusters = 0;
+  }
+  cache[dev].store(clusters > 0 ? clusters : -1, std::memory_order_release);
+  return clusters;
+}
+
+template <int GS>
+cudaError_t launch_pair(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
+                        __half* y, int64_t M, int64_t K, int64_t N, const GemmPlan& p, void* workspace,
+                        cudaStream_t stream) {
+  using L = PairLayout;
+  auto encode = get_encode();
+  if (!encode) return cudaErrorNotSupported;
+  CUtensorMap tx;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)L::kHalfBN};
+    cuuint32_t estr[2] = {1, 1};
+    if (encode(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  static std::atomic<uint64_t> attr_set{0};  // one bit per device that has the attribute
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
+  if (!(attr_set.load(std::memory_order_acquire) >> dev & 1)) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<GS>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set.fetch_or(uint64_t(1) << dev, std::memory_order_acq_rel);
+  }
+  const int64_t NT = (N + kBM - 1) / kBM, T2 = (M + 255) / 256 * ((NT + 1) / 2);
+  int clusters = pair_clusters<GS>(dev);
+  if (clusters <= 0) return launch_bn<256, GS>(x, qweight, scales, zeros, y, M, K, N, p, workspace, stream);
+  if (clusters > T2) clusters = (int)T2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * clusters));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  uint32_t* status = reinterpret_cast<uint32_t*>(workspace);
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<GS>, tx, qweight, scales, zeros, y, (int)M, (int)K, (int)N,
+                            token_tiles_per_block(M, K, 256, 2), status);
+}
+
 template <int GS>
 cudaError_t launch_gs(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
                       __half* y, int64_t M, int64_t K, int64_t N, const GemmPlan& p, void* workspace,
                       cudaStream_t stream) {
+  if (p.pair) return launch_pair<GS>(x, qweight, scales, zeros, y, M, K, N, p, workspace, stream);
   if (p.bn == 256) return launch_bn<256, GS>(x, qweight, scales, zeros, y, M, K, N, p, workspace, stream);
   return launch_bn<128, GS>(x, qweight, scales, zeros, y, M, K, N, p, workspace, stream);
 }
@@ -600,6 +990,9 @@ GemmPlan plan_gemm(int64_t M, int64_t K, int64_t N, int sm_count) {
     p.partial_off = kWsHeaderBytes;
     p.ws_bytes = p.partial_off + (size_t)p.ctas * 2 * p.bn * kBM * sizeof(float);
   }
+  // CTA pairs for the data-parallel schedule at 256-token tiles with at least
+  // two channel tiles
+  p.pair = p.bn == 256 && !p.stream_k && nt >= 2;
   return p;
 }
 
