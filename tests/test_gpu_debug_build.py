@@ -68,12 +68,14 @@ def _pack(W, group):
 
 # (entry point, M, K, N, group): GEMV at M = 1, 2 (integer path), 5, 17 and
 # 32; ragged N and single-k-block K; the GEMM data-parallel with a ragged
-# channel tile, at small M over more tiles than SMs, and stream-K.
+# channel tile, at small M over more tiles than SMs, stream-K, and on CTA
+# pairs (an odd number of channel tiles and a ragged token tile).
 CASES = [("awq_w4a16_gemv", 1, 128, 16, 128), ("awq_w4a16_gemv", 2, 1152, 4096, 128),
          ("awq_w4a16_gemv", 5, 384, 336, 128), ("awq_w4a16_gemv", 17, 4096, 272, 128),
          ("awq_w4a16_gemv", 32, 1024, 592, 64), ("awq_w4a16_gemv", 1, 256, 16656, 32),
          ("awq_w4a16_gemm", 130, 1024, 592, 128), ("awq_w4a16_gemm", 4, 1024, 25600, 128),
-         ("awq_w4a16_gemm", 300, 1024, 9600, 128), ("awq_linear", 40, 1024, 38400, 128)]
+         ("awq_w4a16_gemm", 300, 1024, 9600, 128), ("awq_linear", 40, 1024, 38400, 128),
+         ("awq_w4a16_gemm", 500, 256, 15232, 128)]
 
 
 @pytest.mark.parametrize("fn,M,K,N,group", CASES)
