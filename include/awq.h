@@ -169,7 +169,9 @@ awq_status awq_w4a16_gemv(const void* x, const void* qweight, const void* scales
  * tiles would leave the last wave of SMs short, the k-range of the last tiles
  * is split between CTAs ("stream-K") and a second kernel adds the fp32 parts,
  * which live in the workspace, in a fixed order: results are deterministic
- * for a given device (SM count).
+ * for a given device (SM count). Where whole 256-token tiles are used
+ * without that split (the large prefill shapes), pairs of SMs share each
+ * MMA (clusters of two CTAs, 256 channels x 256 tokens per tile).
  * Source: TinyChat README, New Optimization of Context Stage. */
 awq_status awq_w4a16_gemm(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
                           int64_t M, int64_t K, int64_t N, int group, void* workspace, size_t ws_bytes,

@@ -29,6 +29,9 @@
 //           swizzled, into the A-operand buffer.
 //   warps 11-14 drain a finished accumulator (tcgen05.ld; warp w reads TMEM
 //           lanes 32 (w % 4) ..) into fp16 y and release it.
+// gemm_pair_kernel (below) runs the same roles on clusters of two CTAs that
+// share one MMA stream (tcgen05 cta_group::2) for the data-parallel schedule
+// at 256-token tiles.
 // Rings: x 3 x (BN x 64 k) for BN = 256, 6 x for BN = 128; dequantized weight
 // 3 x (128 x 128 k); packed weight 3 x 8 KiB; each with full/empty mbarriers.
 // (Measured on B200: 3 + 3 stages beat 4 + 2 by ~1 %; two x stages lose 9 %;
