@@ -284,8 +284,9 @@ awq_status awq_get_status_no_alloc(void* stream);
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group);
 
 /* Which kernel awq_linear runs for these sizes on the current device: 1 = the
- * decode GEMV (awq_w4a16_gemv), 2 = the tensor-core GEMM (awq_w4a16_gemm);
- * 0 for M == 0 or invalid sizes. Host only.
+ * decode GEMV (awq_w4a16_gemv), 2 = the tensor-core GEMM (awq_w4a16_gemm) on
+ * one CTA per tile, 3 = the same GEMM on CTA pairs (256-channel x 256-token
+ * tiles); 0 for M == 0 or invalid sizes. Host only.
  * Source: none on the pages (dispatch query). */
 int awq_linear_path(int64_t M, int64_t K, int64_t N, int group);
 

@@ -218,5 +218,18 @@ def test_linear_dispatch_follows_the_measured_split():
     assert awq.awq_linear_path(32, 8192, 57344) == 2   # GEMM
     assert awq.awq_linear_path(0, 4096, 4096) == 0
     assert awq.awq_linear_path(1, 4000, 4096) == 0
+
+
+def test_gemm_runs_on_cta_pairs_for_data_parallel_256_token_tiles():
+    # without a device the library plans for 148 SMs: 256-token tiles without
+    # the stream-K split, and at least two channel tiles, run on CTA pairs
+    assert awq.awq_linear_path(2048, 4096, 28672) == 3   # 1792 tiles, 12.1 waves
+    assert awq.awq_linear_path(8192, 14848, 59392) == 3
+    assert awq.awq_linear_path(500, 256, 15232) == 3     # 119 channel tiles: the last pair has one
+    assert awq.awq_linear_path(512, 4096, 28672) == 2    # stream-K (3.03 waves): one CTA per tile
+    assert awq.awq_linear_path(512, 14336, 4096) == 2    # 128-token tiles
+    assert awq.awq_linear_path(200, 1024, 256) == 2
+    for M, K, N in ((2048, 4096, 28672), (500, 256, 15232)):
+        assert awq.awq_linear_launches(M, K, N) == 1
     assert awq.awq_linear_launches(16, 4096, 28672) == 2   # GEMV + fixup
     assert awq.awq_linear_launches(24, 4096, 28672) == 1   # GEMM, data-parallel

@@ -455,6 +455,7 @@ PAIR_CASES = [(512, 256, 16384, 128), (500, 256, 16512, 128), (512, 256, 16384, 
 
 @pytest.mark.parametrize("M,K,N,group", PAIR_CASES)
 def test_gemm_cta_pairs_match_oracle(M, K, N, group):
+    assert awq.awq_linear_path(M, K, N, group) == 3  # these shapes run on CTA pairs
     W, dev, hp = _packed(N, K, f"pair{K}x{N}", group=group)
     x = awq_synth.matrix_f16(awq_synth.key(0, 96, f"pair{K}x{N}/x{M}"), M, K, 1.0)
     xd = to_dev(x.view(np.uint16), torch.float16)

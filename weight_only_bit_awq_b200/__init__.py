@@ -275,7 +275,8 @@ def awq_linear_launches(M: int, K: int, N: int, group: int = GROUP) -> int:
 
 
 def awq_linear_path(M: int, K: int, N: int, group: int = GROUP) -> int:
-    """Kernel awq_linear runs for these sizes: 1 = the GEMV, 2 = the GEMM, 0 = none."""
+    """Kernel awq_linear runs for these sizes: 1 = the GEMV, 2 = the GEMM, 3 = the
+    GEMM on CTA pairs, 0 = none."""
     return int(lib.awq_linear_path(M, K, N, group))
 
 

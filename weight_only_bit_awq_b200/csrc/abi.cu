@@ -332,7 +332,9 @@ awq_status awq_w4a8_gemm(const void* x8, const void* sx, const void* qweight, co
 
 int awq_linear_path(int64_t M, int64_t K, int64_t N, int group) {
   if (M <= 0 || M > kMaxM || check_kn(K, N, group) != AWQ_OK) return 0;
-  return linear_uses_gemv(M, N, sm_count_or_default()) ? 1 : 2;
+  const int sms = sm_count_or_default();
+  if (linear_uses_gemv(M, N, sms)) return 1;
+  return plan_gemm(M, K, N, sms).pair ? 3 : 2;
 }
 
 int awq_linear_launches(int64_t M, int64_t K, int64_t N, int group) {
