@@ -126,6 +126,92 @@ __device__ __forceinline__ void tile_coords(int t, int MT, int NT, int GM, int& 
   nt = w / gb;
 }
 
+// ---- pieces shared by gemm_kernel and gemm_pair_kernel ----
+
+// Fill code stage `st` (one lane-0 thread of the producer warp issues the
+// bulk copy; the warp's lanes copy the scale and zero rows): the R <= 8 row
+// blocks of channel tile gi for k-block kb are one contiguous run of R KiB in
+// the packed layout (qbytes = R KiB, 0 for a channel tile past N). The tile's
+// scale and zero-point rows of the k-block follow by cp.async; the stage's
+// barrier `full` counts the bytes plus one arrival per lane.
+template <int GS>
+__device__ __forceinline__ void fill_code_stage(uint32_t st, uint32_t full, const uint32_t* __restrict__ qweight,
+                                                const __half* __restrict__ scales, const uint8_t* __restrict__ zeros,
+                                                int64_t gi, int kb, int KB, int64_t NB, int n0, int K, int N,
+                                                uint32_t qbytes, int lane, uint32_t* status) {
+  constexpr int kGPK = kKPerBlock / GS;
+  const int64_t qw0 = qbytes > 0 ? unit_first_block(gi, kb, KB, NB) * kWordsPerBlock : 0;
+  const bool qok = qbytes > 0 && AWQ_CHECK(in_range(qw0, qbytes / 4, (int64_t)K * N / 8), status);
+  if (lane == 0) ptx::mbar_arrive_expect_tx(full, qok ? qbytes : 0u);
+  __syncwarp();
+  if (lane == 0 && qok) ptx::bulk_g2s(st, qweight + qw0, qbytes, full);
+  for (int p = lane; p < kGPK * 16; p += 32) {  // kGPK rows of 128 scales: 16 B = 8 output channels
+    const int g = p >> 4, l = p & 15;
+    if (n0 + 8 * l < N &&
+        AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * N + n0 + 8 * l, 8, (int64_t)(K / GS) * N), status))
+      ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
+  }
+  for (int p = lane; p < kGPK * 8; p += 32) {  // kGPK rows of 64 zero bytes: 8 B = 16 output channels
+    const int g = p >> 3, l = p & 7;
+    if (n0 + 16 * l < N &&
+        AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l, 8, (int64_t)(K / GS) * (N / 2)),
+                  status))
+      ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l, zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
+  }
+  ptx::cp_async_arrive_noinc(full);
+}
+
+// One weight row's codes, scales and zero points of a k-block, read from a
+// code stage by the row's dequant thread. It reads the row's 64 B of codes as
+// four 16-byte chunks in an order rotated by rot = (row / 2) % 4, so that
+// every 8-lane phase of the shared loads (and of the swizzled stores below)
+// touches distinct banks. Rows past N read stale values: their outputs are
+// never stored.
+template <int GS>
+struct RowCodes {
+  uint4 c[4];                                         // c[jj] holds words 4 ((jj + rot) & 3) ..
+  uint32_t s[kKPerBlock / GS], z[kKPerBlock / GS];  // fp16 bits of the scale, zero point, per group
+};
+template <int GS>
+__device__ __forceinline__ void load_row_codes(const uint8_t* qst, int row, int rot, RowCodes<GS>& rc) {
+  const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64;
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) rc.c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 3));
+#pragma unroll
+  for (int g = 0; g < kKPerBlock / GS; ++g) {
+    rc.s[g] = reinterpret_cast<const uint16_t*>(qst + kQScaleOff + 256 * g)[row];
+    rc.z[g] = (qst[kQZeroOff + 64 * g + (row >> 1)] >> (4 * (row & 1))) & 0xF;
+  }
+}
+// fp16_rne((q - z) s) of the row's 128 inputs into its 128-byte line `wt` of
+// each 64-k half of an A buffer (K-major, 128-byte swizzle).
+template <int GS>
+__device__ __forceinline__ void store_row_dequant(uint8_t* wt, int row, int rot, const RowCodes<GS>& rc) {
+  constexpr int kGPK = kKPerBlock / GS, J = GS / 32;
+  __half2 s2[kGPK], zlo[kGPK], zhi[kGPK];
+#pragma unroll
+  for (int g = 0; g < kGPK; ++g) {
+    // fp16 bit patterns: s itself, 1024 + z = 0x6400 + z, -(64 + z) = 0xD400 + 16 z
+    s2[g] = u2h(rc.s[g] * 0x00010001u);
+    zlo[g] = u2h((0x6400u + rc.z[g]) * 0x00010001u);
+    zhi[g] = u2h((0xD400u + (rc.z[g] << 4)) * 0x00010001u);
+  }
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    const int cj = (jj + rot) & 3;  // rc.c[jj] holds words 4 cj .. 4 cj + 3 of the row
+    const uint32_t words[4] = {rc.c[jj].x, rc.c[jj].y, rc.c[jj].z, rc.c[jj].w};
+#pragma unroll
+    for (int ww = 0; ww < 4; ++ww) {
+      // word 4 cj + ww holds inputs k0 .. k0 + 7 of group ww / J (word_k0
+      // written out for this word: ww is a constant here)
+      const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
+      const int chunk = (k0 & 63) >> 3;  // 16-byte chunk (8 k) within the 64-k half
+      uint8_t* dst = wt + (k0 >> 6) * kWHalfBytes;
+      *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) = dequant_word(words[ww], zlo[g], zhi[g], s2[g]);
+    }
+  }
+}
+
 // GS: group size (128, 64 or 32), kGPK = 128 / GS groups per k-block.
 // Persistent: CTA c computes the whole tiles c, c + P, c + 2P, ... below Tdp
 // (P = gridDim.x; tile t maps to (token tile, channel tile) by tile_coords, so
@@ -235,10 +321,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kWarpQ) {
     // ---------------- packed-weight producer ----------------
-    // The R <= 8 row blocks of a tile's group are one contiguous run of
-    // R KiB per k-block in the packed layout: one 1-D bulk copy each. The
-    // tile's scale and zero-point rows of the k-block follow by cp.async.
-    constexpr int kGPK = kKPerBlock / GS;
     const int64_t NB = N / kRowsPerBlock;
     int i = 0;
     bool ok = true;
@@ -246,34 +328,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t, kb0, kb1, mt, nt;
       seg(j, t, kb0, kb1);
       tile_mn(t, mt, nt);
-      const int64_t gi = nt;
-      const int n0 = (int)gi * kBM;
-      const uint32_t qbytes = (uint32_t)(group_rows(gi, NB) * 1024);
+      const uint32_t qbytes = (uint32_t)(group_rows(nt, NB) * 1024);
       for (int kb = kb0; kb < kb1; ++kb, ++i) {
         const int s = i % kQStages;
         if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((i / kQStages) & 1) ^ 1, abort_flag, status);
         if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
-        const uint32_t st = sbase + L::kQOff + s * kQStride;
-        const int64_t qw0 = unit_first_block(gi, kb, KB, NB) * kWordsPerBlock;
-        const bool qok = AWQ_CHECK(in_range(qw0, qbytes / 4, (int64_t)K * N / 8), status);
-        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qok ? qbytes : 0u);
-        __syncwarp();
-        if (lane == 0 && qok) ptx::bulk_g2s(st, qweight + qw0, qbytes, bar(kBarQFull + s));
-        for (int p = lane; p < kGPK * 16; p += 32) {  // kGPK rows of 128 scales: 16 B = 8 output channels
-          const int g = p >> 4, l = p & 15;
-          if (n0 + 8 * l < N &&
-              AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * N + n0 + 8 * l, 8, (int64_t)(K / GS) * N), status))
-            ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
-        }
-        for (int p = lane; p < kGPK * 8; p += 32) {  // kGPK rows of 64 zero bytes: 8 B = 16 output channels
-          const int g = p >> 3, l = p & 7;
-          if (n0 + 16 * l < N &&
-              AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l, 8, (int64_t)(K / GS) * (N / 2)),
-                        status))
-            ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l,
-                            zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
-        }
-        ptx::cp_async_arrive_noinc(bar(kBarQFull + s));
+        fill_code_stage<GS>(sbase + L::kQOff + s * kQStride, bar(kBarQFull + s), qweight, scales, zeros, nt, kb, KB, NB,
+                            nt * kBM, K, N, qbytes, lane, status);
       }
     }
     if (!ok && lane == 0)
@@ -323,14 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- dequantize ----------------
     // Two groups of four warps take alternate k-blocks, so two k-blocks are
     // in flight and one group's barrier waits, loads and proxy fence overlap
-    // the other's arithmetic. In a group, thread = weight row: it reads the
-    // row's 64 B of codes as four 16-byte chunks in an order rotated by
-    // (row / 2) % 4, so that every 8-lane phase of the shared loads and of the
-    // swizzled stores touches distinct banks.
+    // the other's arithmetic; in a group, thread = weight row.
     const int d = threadIdx.x - kFirstDeqWarp * 32;  // 0..255
     const int grp = d >> 7, row = d & (kBM - 1);
     const int rot = (row >> 1) & 3;
-    constexpr int kGPK = kKPerBlock / GS;
     bool ok = true;
     int i = 0;  // k-blocks so far (Q and W stage uses)
     for (int j = 0; j < nseg && ok; ++j) {
@@ -345,48 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // wait cannot tell those phases apart)
         const int qs = i % kQStages;
         if (!(ok = wait_bar(bar(kBarQFull + qs), (i / kQStages) & 1, abort_flag, status))) break;
-        const uint8_t* qst = smem + L::kQOff + qs * kQStride;
-        const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64;
-        uint4 c[4];
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 3));
-        // fp16 bits of the scale and the zero point of this row, per group (rows
-        // past N read stale values: their outputs are never stored)
-        uint32_t s[kGPK], z[kGPK];
-#pragma unroll
-        for (int g = 0; g < kGPK; ++g) {
-          s[g] = reinterpret_cast<const uint16_t*>(qst + kQScaleOff + 256 * g)[row];
-          z[g] = (qst[kQZeroOff + 64 * g + (row >> 1)] >> (4 * (row & 1))) & 0xF;
-        }
+        RowCodes<GS> rc;
+        load_row_codes<GS>(smem + L::kQOff + qs * kQStride, row, rot, rc);
         ptx::mbar_arrive(bar(kBarQEmpty + qs));
-
         const int ws = i % kWStages;
         if (!(ok = wait_bar(bar(kBarWEmpty + ws), ((i / kWStages) & 1) ^ 1, abort_flag, status))) break;
-        __half2 s2[kGPK], zlo[kGPK], zhi[kGPK];
-#pragma unroll
-        for (int g = 0; g < kGPK; ++g) {
-          // fp16 bit patterns: s itself, 1024 + z = 0x6400 + z, -(64 + z) = 0xD400 + 16 z
-          s2[g] = u2h(s[g] * 0x00010001u);
-          zlo[g] = u2h((0x6400u + z[g]) * 0x00010001u);
-          zhi[g] = u2h((0xD400u + (z[g] << 4)) * 0x00010001u);
-        }
-        uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int cj = (jj + rot) & 3;  // c[jj] holds words 4 cj .. 4 cj + 3 of the row
-          const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
-#pragma unroll
-          for (int ww = 0; ww < 4; ++ww) {
-            // word 4 cj + ww holds inputs k0 .. k0 + 7 of group ww / (GS / 32)
-            // (word_k0 written out for this word: ww is a constant here)
-            constexpr int J = GS / 32;
-            const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
-            const int chunk = (k0 & 63) >> 3;  // 16-byte chunk (8 k) within the 64-k half
-            uint8_t* dst = wt + (k0 >> 6) * kWHalfBytes;
-            *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) =
-                dequant_word(words[ww], zlo[g], zhi[g], s2[g]);
-          }
-        }
+        store_row_dequant<GS>(smem + L::kWOff + ws * kWBytes + row * 128, row, rot, rc);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(bar(kBarWFull + ws));
       }
@@ -577,42 +598,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kWarpQ) {
     // ---------------- packed-weight producer (this CTA's channel tile) ----------------
-    constexpr int kGPK = kKPerBlock / GS;
     const int64_t NB = N / kRowsPerBlock;
     int i = 0;
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
       int mt, nt;
       tile(j, mt, nt);
-      const bool has = nt < NT;
-      const int64_t gi = nt;
-      const int n0 = nt * kBM;
-      const uint32_t qbytes = has ? (uint32_t)(group_rows(gi, NB) * 1024) : 0u;
+      const uint32_t qbytes = nt < NT ? (uint32_t)(group_rows(nt, NB) * 1024) : 0u;
       for (int kb = 0; kb < KB; ++kb, ++i) {
         const int s = i % kQStages;
         if (lane == 0) ok = wait_bar(bar(kBarQEmpty + s), ((i / kQStages) & 1) ^ 1, abort_flag, status);
         if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
-        const uint32_t st = sbase + L::kQOff + s * kQStride;
-        const int64_t qw0 = has ? unit_first_block(gi, kb, KB, NB) * kWordsPerBlock : 0;
-        const bool qok = qbytes > 0 && AWQ_CHECK(in_range(qw0, qbytes / 4, (int64_t)K * N / 8), status);
-        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kBarQFull + s), qok ? qbytes : 0u);
-        __syncwarp();
-        if (lane == 0 && qok) ptx::bulk_g2s(st, qweight + qw0, qbytes, bar(kBarQFull + s));
-        for (int p = lane; p < kGPK * 16; p += 32) {
-          const int g = p >> 4, l = p & 15;
-          if (n0 + 8 * l < N &&
-              AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * N + n0 + 8 * l, 8, (int64_t)(K / GS) * N), status))
-            ptx::cp_async_16(st + kQScaleOff + 256 * g + 16 * l, scales + ((int64_t)kb * kGPK + g) * N + n0 + 8 * l);
-        }
-        for (int p = lane; p < kGPK * 8; p += 32) {
-          const int g = p >> 3, l = p & 7;
-          if (n0 + 16 * l < N &&
-              AWQ_CHECK(in_range(((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l, 8, (int64_t)(K / GS) * (N / 2)),
-                        status))
-            ptx::cp_async_8(st + kQZeroOff + 64 * g + 8 * l,
-                            zeros + ((int64_t)kb * kGPK + g) * (N / 2) + n0 / 2 + 8 * l);
-        }
-        ptx::cp_async_arrive_noinc(bar(kBarQFull + s));
+        fill_code_stage<GS>(sbase + L::kQOff + s * kQStride, bar(kBarQFull + s), qweight, scales, zeros, nt, kb, KB, NB,
+                            nt * kBM, K, N, qbytes, lane, status);
       }
     }
     if (!ok && lane == 0)
@@ -661,7 +659,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int d = threadIdx.x - kFirstDeqWarp * 32;
     const int grp = d >> 7, row = d & (kBM - 1);
     const int rot = (row >> 1) & 3;
-    constexpr int kGPK = kKPerBlock / GS;
     bool ok = true;
     int i = 0;
     for (int j = 0; j < ntiles && ok; ++j) {
@@ -669,43 +666,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((i & 1) != grp) continue;
         const int qs = i % kQStages;
         if (!(ok = wait_bar(bar(kBarQFull + qs), (i / kQStages) & 1, abort_flag, status))) break;
-        const uint8_t* qst = smem + L::kQOff + qs * kQStride;
-        const uint8_t* qrow = qst + (row >> 4) * 1024 + (row & 15) * 64;
-        uint4 c[4];
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) c[jj] = *reinterpret_cast<const uint4*>(qrow + 16 * ((jj + rot) & 3));
-        uint32_t s[kGPK], z[kGPK];
-#pragma unroll
-        for (int g = 0; g < kGPK; ++g) {
-          s[g] = reinterpret_cast<const uint16_t*>(qst + kQScaleOff + 256 * g)[row];
-          z[g] = (qst[kQZeroOff + 64 * g + (row >> 1)] >> (4 * (row & 1))) & 0xF;
-        }
+        RowCodes<GS> rc;
+        load_row_codes<GS>(smem + L::kQOff + qs * kQStride, row, rot, rc);
         ptx::mbar_arrive(bar(kBarQEmpty + qs));
-
         const int ws = i % kWStages;
         if (!(ok = wait_bar(bar(kBarWEmpty + ws), ((i / kWStages) & 1) ^ 1, abort_flag, status))) break;
-        __half2 s2[kGPK], zlo[kGPK], zhi[kGPK];
-#pragma unroll
-        for (int g = 0; g < kGPK; ++g) {
-          s2[g] = u2h(s[g] * 0x00010001u);
-          zlo[g] = u2h((0x6400u + z[g]) * 0x00010001u);
-          zhi[g] = u2h((0xD400u + (z[g] << 4)) * 0x00010001u);
-        }
-        uint8_t* wt = smem + L::kWOff + ws * kWBytes + row * 128;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int cj = (jj + rot) & 3;
-          const uint32_t words[4] = {c[jj].x, c[jj].y, c[jj].z, c[jj].w};
-#pragma unroll
-          for (int ww = 0; ww < 4; ++ww) {
-            constexpr int J = GS / 32;
-            const int k0 = GS * (ww / J) + 8 * (cj * J + ww % J), g = ww / J;
-            const int chunk = (k0 & 63) >> 3;
-            uint8_t* dst = wt + (k0 >> 6) * kWHalfBytes;
-            *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) =
-                dequant_word(words[ww], zlo[g], zhi[g], s2[g]);
-          }
-        }
+        store_row_dequant<GS>(smem + L::kWOff + ws * kWBytes + row * 128, row, rot, rc);
         ptx::fence_proxy_async_smem();
         if (leader)
           ptx::mbar_arrive(bar(kBarWFull + ws));
