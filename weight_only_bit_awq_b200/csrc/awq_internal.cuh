@@ -3,6 +3,7 @@
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include "awq.h"
@@ -82,6 +83,9 @@ struct DeviceInfo {
   size_t smem_optin = 0;
 };
 const DeviceInfo& device_info();   // current device
+
+// The driver's cuTensorMapEncodeTiled (looked up once; nullptr if missing).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // GEMV launch plan (shared by awq_workspace_bytes and the launcher).
 struct GemvPlan {

@@ -520,25 +520,12 @@ int token_tiles_per_block(int64_t M, int64_t K, int BN, int xbytes) {
   return (int)(g < mt ? g : mt);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 template <int BN, int GS>
 cudaError_t launch_bn(const uint8_t* x8, const float* sx, const uint32_t* qweight, const __half* scales,
                       const uint8_t* zeros, const int8_t* row_exp, __half* y, int64_t M, int64_t K, int64_t N,
                       uint32_t* status, cudaStream_t stream) {
   using L = Layout<BN>;
-  auto encode = get_encode();
+  auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap tx;
   {

@@ -778,25 +778,12 @@ int token_tiles_per_block(int64_t M, int64_t K, int BN, int xbytes) {
   return (int)(g < mt ? g : mt);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 template <int BN, int GS>
 cudaError_t launch_bn(const __half* x, const uint32_t* qweight, const __half* scales, const uint8_t* zeros,
                       __half* y, int64_t M, int64_t K, int64_t N, const GemmPlan& p, void* workspace,
                       cudaStream_t stream) {
   using L = Layout<BN>;
-  auto encode = get_encode();
+  auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap tx;
   {
@@ -870,7 +857,7 @@ cudaError_t launch_pair(const __half* x, const uint32_t* qweight, const __half* 
                         __half* y, int64_t M, int64_t K, int64_t N, const GemmPlan& p, void* workspace,
                         cudaStream_t stream) {
   using L = PairLayout;
-  auto encode = get_encode();
+  auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap tx;
   {
