@@ -10,7 +10,9 @@ GPU by awq_pack before timing. Eight rotating copies of the packed weights
 (8 x 105 MB, more than the 126 MB L2) make every step read HBM. The eight
 steps that use them one after another are captured in one CUDA graph, the way
 a decode step of a whole model (many decoder layers) is one graph: the graph
-launch boundary (about 5 us, measured) is paid once per eight steps.
+launch boundary (about 5 us, measured) is paid once per graph. Up to 64 timed
+steps run as one graph of exactly that many steps (step i on copy i mod 8);
+longer runs replay the eight-step graph.
 
 Prints ONE JSON line (rank 0): the metric (GB/s of algorithmic bytes, whole
 job), the roofline of the GEMV kernel, an end-to-end figure through the
@@ -474,28 +476,34 @@ def run_ours(args):
         for L, x, y, (qw, sc, ze) in zip(layers, xs, ys, packed[r]):
             awq.awq_linear(x, qw, sc, ze, L.N, ws, y=y)
 
-    # CUDA graphs: graphs[j] holds j consecutive steps (weight copies 0 ..
-    # j - 1, 4 layers each); k steps replay graphs[ROTATIONS] k // ROTATIONS
+    # CUDA graphs: graphs[j] holds j consecutive steps (step i on weight copy
+    # i % ROTATIONS, 4 layers each). Up to WHOLE_GRAPH_STEPS steps run as one
+    # graph of exactly k steps; more replay graphs[ROTATIONS] k // ROTATIONS
     # times, then graphs[k % ROTATIONS] once
+    WHOLE_GRAPH_STEPS = 64
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
         for r in range(ROTATIONS):   # warm the launch paths before capture
             step(r)
     torch.cuda.synchronize()
+
+    def plan(k):
+        return [k] if k <= WHOLE_GRAPH_STEPS else [ROTATIONS] * (k // ROTATIONS) + (
+            [k % ROTATIONS] if k % ROTATIONS else [])
+
     graphs = {}
-    for j in {ROTATIONS, args.steps % ROTATIONS, args.warmup % ROTATIONS} - {0}:
+    for j in set(plan(args.steps) + plan(args.warmup)) - {0}:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            for r in range(j):
-                step(r)
+            for i in range(j):
+                step(i % ROTATIONS)
         graphs[j] = g
     torch.cuda.synchronize()
 
     def run_steps(k):  # exactly k steps
-        for _ in range(k // ROTATIONS):
-            graphs[ROTATIONS].replay()
-        if k % ROTATIONS:
-            graphs[k % ROTATIONS].replay()
+        for j in plan(k):
+            if j:
+                graphs[j].replay()
 
     # every graph the warm-up and the timed region use is replayed once first,
     # so neither region holds a graph's first launch
@@ -685,9 +693,11 @@ def run_ours(args):
                    "layers": [[L.name, L.K, L.N] for L in layers],
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"{ROTATIONS} rotating packed-weight copies ({ROTATIONS * step_bytes / 1e6:.0f} MB > 126 MB L2)",
-                   "timing": f"CUDA graphs of {ROTATIONS} consecutive steps (one per weight copy) and one graph "
-                             f"of the remaining steps, each replayed once before warm-up; CUDA events on the "
-                             f"replay stream"},
+                   "timing": (f"one CUDA graph of all {args.steps} steps (step i on weight copy i mod "
+                              f"{ROTATIONS})" if args.steps <= WHOLE_GRAPH_STEPS else
+                              f"CUDA graphs of {ROTATIONS} consecutive steps (one per weight copy) and one graph "
+                              f"of the remaining steps") + ", each replayed once before warm-up; CUDA events on "
+                                                          "the replay stream"},
         "roofline": {"bound": "hbm", "achieved": per_gpu_gbs, "peak": hbm, "unit": "GB/s",
                      "frac": per_gpu_gbs / hbm, "traffic": traffic,
                      "kernel": "gemv_kernel (awq_w4a16_gemv via awq_linear)",
