@@ -166,6 +166,12 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
     // unit within the group), one for the activations (unit within the group).
     int64_t cgi = u0 / rg.UPG;
     int cj = (int)(u0 % rg.UPG), xj = cj;
+    // L2 policies: the codes, scales and zeros are read once, so their lines
+    // go first; x is read by every CTA that shares its k-range, so it stays.
+    // The previous layer's partial sums, y and the next layer's x then stay
+    // in L2 while the weights stream past them.
+    const uint64_t pol_stream = ptx::l2_policy_evict_first();
+    const uint64_t pol_x = ptx::l2_policy_evict_last();
     auto issue_codes = [&](int s) {  // codes, scales, zeros of the next unit into stage s; arms it
       const int R = (int)group_rows(cgi, rg.NB);
       const int64_t kb0 = (int64_t)cj * KU;
@@ -179,7 +185,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
         ptx::mbar_arrive_expect_tx(full(s),
                                    (uint32_t)((qok ? ku * R * 1024 : 0) + (kXWarp ? 0 : M * ku * kXRowBytes)));
       __syncwarp();
-      if (lane == 0 && qok) ptx::bulk_g2s(st + L.q, qweight + qw0, (uint32_t)(ku * R * 1024), full(s));
+      if (lane == 0 && qok)
+        ptx::bulk_g2s_hint(st + L.q, qweight + qw0, (uint32_t)(ku * R * 1024), full(s), pol_stream);
       const __half* srow = scales + kb0 * kGPK * N + kGroupBlocks * kRowsPerBlock * cgi;
       for (int p = lane; p < ku * kGPK * 16; p += 32) {  // ku * kGPK rows of 32 R bytes
         const int j = p >> 4, l = p & 15;
@@ -188,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
                                (int64_t)(K / GS) * N) &&
                           in_range(s * L.bytes + L.s + j * kKbScaleBytes + 16 * l, 16, dynamic_smem_bytes()),
                       status))
-          ptx::cp_async_16(st + L.s + j * kKbScaleBytes + 16 * l, srow + (int64_t)j * N + 8 * l);
+          ptx::cp_async_16_hint(st + L.s + j * kKbScaleBytes + 16 * l, srow + (int64_t)j * N + 8 * l,
+                                pol_stream);
       }
       const uint8_t* zrow = zeros + kb0 * kGPK * (N / 2) + 64 * cgi;
       for (int p = lane; p < ku * kGPK * 8; p += 32) {  // ku * kGPK rows of 8 R bytes
@@ -198,7 +206,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
                                (int64_t)(K / GS) * (N / 2)) &&
                           in_range(s * L.bytes + L.z + j * kKbZeroBytes + 8 * l, 8, dynamic_smem_bytes()),
                       status))
-          ptx::cp_async_8(st + L.z + j * kKbZeroBytes + 8 * l, zrow + (int64_t)j * (N / 2) + 8 * l);
+          ptx::cp_async_8_hint(st + L.z + j * kKbZeroBytes + 8 * l, zrow + (int64_t)j * (N / 2) + 8 * l,
+                               pol_stream);
       }
       ptx::cp_async_arrive_noinc(full(s));
       if (++cj == rg.UPG) {
@@ -220,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2)
         if (AWQ_CHECK(in_range((int64_t)lane * K + kb0 * kKPerBlock, (int64_t)ku * kKPerBlock, (int64_t)M * K) &&
                           in_range(s * L.bytes + L.x + L.xrow * lane, ku * kXRowBytes, dynamic_smem_bytes()),
                       status))
-          ptx::bulk_g2s(sbase + s * L.bytes + L.x + L.xrow * lane, x + (int64_t)lane * K + kb0 * kKPerBlock,
-                        (uint32_t)(ku * kXRowBytes), xb);
+          ptx::bulk_g2s_hint(sbase + s * L.bytes + L.x + L.xrow * lane, x + (int64_t)lane * K + kb0 * kKPerBlock,
+                             (uint32_t)(ku * kXRowBytes), xb, pol_x);
 #ifdef AWQ_DEBUG
         else
           asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(xb), "r"((uint32_t)(ku * kXRowBytes))
