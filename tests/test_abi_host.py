@@ -103,6 +103,18 @@ def test_gemm_schedule_on_148_sms():
     assert awq.awq_linear_launches(40, 128, 1024, 128) == 1
 
 
+def test_gemv_launches_no_fixup_when_every_cta_range_ends_on_a_group():
+    # 148 SMs, M = 1: at K = 512 a group of 128 channels is one unit of 4
+    # k-blocks, so N = 148 x 128 (148 units on 148 CTAs) and N = 296 x 128
+    # (296 on 296) give every CTA whole groups: no split row, no fixup kernel
+    assert awq.awq_linear_launches(1, 512, 148 * 128) == 1
+    assert awq.awq_linear_launches(1, 512, 296 * 128) == 1
+    # K = 1024 (2 units per group over 296 CTAs) and K = 4096 (8 per group
+    # over 256 CTAs) put CTA boundaries inside groups: the GEMV and its fixup
+    assert awq.awq_linear_launches(1, 1024, 148 * 128) == 2
+    assert awq.awq_linear_launches(1, 4096, 4096) == 2
+
+
 def _linear(fn, x=FAKE, q=FAKE2, s=FAKE3, z=FAKE4, y=FAKE5, M=1, K=4096, N=4096, group=128, ws=FAKE6,
             ws_bytes=1 << 30):
     return getattr(L, fn)(x, q, s, z, y, M, K, N, group, ws, ws_bytes, None)
