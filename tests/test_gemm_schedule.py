@@ -15,7 +15,10 @@ This module models that schedule in Python and checks
 - that every (tile, k-block) is computed exactly once, that a CTA's partial
   segments are its first (slot 0) and last (slot 1) stream-K segments, and that
   the fixup finds each contributor's part where it was written, for many shapes
-  and SM counts.
+  and SM counts;
+- that the grouped tile order visits every tile once (ragged last block
+  included), and that the CTA-pair schedule computes every output tile once,
+  the channel tile past the last only on the second CTA of the last pair.
 """
 import pytest
 
@@ -107,3 +110,56 @@ def test_the_library_plans_the_same_schedule():
         slots = 148 * 2 * p["bn"] * 128 * 4 if p["sk"] else 0
         assert awq.awq_workspace_bytes(M, K, N) == 256 + slots, (M, K, N)
     assert seen == {True, False}
+
+
+# ---- tile order and the CTA-pair schedule ----
+# Tiles t = 0 .. MT x NT - 1 map to (token tile, channel tile) in blocks of GM
+# token tiles (the last block may hold fewer); within a block the token tile
+# runs fastest, so the CTAs working at the same time share a few weight tiles.
+# The CTA-pair kernel walks pair tiles (token tile, channel-tile pair np) in
+# that order with NP = ceil(NT / 2) in place of NT: cluster cl of P2 takes pair
+# tiles cl, cl + P2, ...; the pair's CTA of rank r computes channel tile
+# 2 np + r, which is past the last when NT is odd (that CTA only takes part in
+# the pair's MMAs).
+
+
+def tile_coords(t, MT, NT, GM):
+    blk, w = t // (GM * NT), t % (GM * NT)
+    gb = min(GM, MT - blk * GM)
+    return blk * GM + w % gb, w // gb
+
+
+def gm_of(M, K, BN):
+    """Token tiles per block: the block's x within ~48 MB of L2, at least one."""
+    return max(1, min((48 << 20) // (BN * K * 2), cdiv(M, BN)))
+
+
+def test_the_tile_order_visits_every_tile_once():
+    for MT in range(1, 13):
+        for NT in range(1, 13):
+            for GM in range(1, MT + 1):
+                seen = [tile_coords(t, MT, NT, GM) for t in range(MT * NT)]
+                assert sorted(seen) == [(m, n) for m in range(MT) for n in range(NT)], (MT, NT, GM)
+
+
+@pytest.mark.parametrize("M,K,N", [(2048, 4096, 28672), (8192, 14848, 59392), (500, 256, 15232), (257, 128, 272),
+                                   (4096, 14336, 4096), (1024, 2048, 16 * 128 * 3)])
+@pytest.mark.parametrize("P2", [1, 3, 74, 148])
+def test_cta_pairs_compute_every_output_tile_once(M, K, N, P2):
+    MT, NT = cdiv(M, 256), cdiv(N, 128)
+    NP = cdiv(NT, 2)
+    T2 = MT * NP
+    GM = gm_of(M, K, 256)
+    done = {}
+    for cl in range(P2):
+        ntiles = (T2 - 1 - cl) // P2 + 1 if cl < T2 else 0
+        for j in range(ntiles):
+            mt, np_ = tile_coords(cl + j * P2, MT, NP, GM)
+            for rank in (0, 1):
+                nt = 2 * np_ + rank
+                if nt >= NT:
+                    assert NT % 2 == 1 and np_ == NP - 1 and rank == 1
+                    continue
+                assert (mt, nt) not in done
+                done[(mt, nt)] = (cl, rank)
+    assert sorted(done) == [(m, n) for m in range(MT) for n in range(NT)]
