@@ -50,7 +50,8 @@
  * Conventions for every entry point
  * ---------------------------------------------------------------------------
  *   Shapes     M >= 0 (M = 0 is a no-op), K > 0 and K % 128 == 0, N > 0 and
- *              N % 16 == 0, group 128, 64 or 32 (else AWQ_ERR_UNSUPPORTED).
+ *              N % 16 == 0 (else AWQ_ERR_SHAPE); group 128, 64 or 32, and
+ *              K, N <= 2^22, M <= 2^24 (else AWQ_ERR_UNSUPPORTED).
  *   Pointers   device pointers unless stated; all non-null (x and y may be
  *              null when M == 0) and 16-byte aligned (AWQ_ERR_INVALID_ARG /
  *              AWQ_ERR_ALIGNMENT). Outputs may not overlap inputs.

@@ -130,6 +130,8 @@ def test_linear_argument_errors(fn):
     assert _linear(fn, N=4104) == awq.AWQ_ERR_SHAPE
     assert _linear(fn, group=256) == awq.AWQ_ERR_UNSUPPORTED
     assert _linear(fn, group=96) == awq.AWQ_ERR_UNSUPPORTED
+    assert _linear(fn, K=1 << 23) == awq.AWQ_ERR_UNSUPPORTED              # K, N <= 2^22
+    assert _linear(fn, N=1 << 23) == awq.AWQ_ERR_UNSUPPORTED
     assert _linear(fn, x=None) == awq.AWQ_ERR_INVALID_ARG
     assert _linear(fn, y=None) == awq.AWQ_ERR_INVALID_ARG
     assert _linear(fn, ws=None) == awq.AWQ_ERR_INVALID_ARG
@@ -143,6 +145,11 @@ def test_linear_argument_errors(fn):
 
 def test_gemv_rejects_large_batches():
     assert _linear("awq_w4a16_gemv", M=33) == awq.AWQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("fn", ["awq_w4a16_gemm", "awq_linear"])
+def test_batches_above_the_limit_are_rejected(fn):
+    assert _linear(fn, M=(1 << 24) + 1) == awq.AWQ_ERR_UNSUPPORTED         # M <= 2^24
 
 
 def test_pack_and_dequant_argument_errors():
